@@ -1,0 +1,559 @@
+#!/usr/bin/env python
+"""Benchmark of the attention hot path on B200; prints ONE JSON line (rank 0).
+
+Headline workload: the Whisper-large-shaped decoder cross-attention decode step -- 64 requests
+x 1 query token over 1500-token encoder contexts, 20/20 heads, head_dim 64, pages of 16 tokens
+scattered over a 16384-page pool.  One step is what a decoder step of that model does with
+this path: one plan (host, once per step) and then one layer call per decoder layer (32),
+each layer reading its own layer's context pool.  All pools stay resident in HBM (32 x 2 x
+671 MB); every layer's 491.5 MB of valid K/V exceeds the 126 MB L2, so nothing is served
+from L2 between layers.
+
+  value  KV HBM GB/s of the whole step: algorithmic bytes (valid K/V once per KV head + Q + O)
+         over the device time of K steps (CUDA events, max over ranks).
+  e2e    the same metric through the public API with host buffers: every layer's q is copied
+         host->device from pinned memory and every output back, inside the timed region.
+
+The other four workloads (tiny decode, packed multi-token, ragged block-causal, long-context
+split-KV) are measured per layer call under "workloads".  `--impl reference` times the CPU
+float64 oracle (the only reference this path has) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+LAYERS = 32                       # decoder layers of the Whisper-large shape
+SPEC_TC_TFLOPS = 2250.0           # dense bf16 per B200 (nominal)
+SPEC_HBM_GBS = 8000.0             # HBM3e per B200 (nominal)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--skip-workloads", action="store_true",
+                    help="only the headline workload (no per-workload table)")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------- work accounting
+
+def paged_work(case):
+    """(flops, bytes) of one layer call: 4*d*Hq per visible (query, key) pair; valid K/V read
+    once per KV head, plus Q and O."""
+    q_len = np.diff(case.qo_indptr).astype(np.int64)
+    kv = case.kv_len.astype(np.int64)
+    pairs = int((q_len * kv).sum())
+    flops = 4 * case.head_dim * case.num_qo_heads * pairs
+    kv_tokens = int(kv[q_len > 0].sum())
+    kv_bytes = kv_tokens * case.num_kv_heads * case.head_dim * 2 * 2
+    qo_bytes = int(q_len.sum()) * case.num_qo_heads * case.head_dim * 2 * 2
+    return flops, kv_bytes + qo_bytes, kv_bytes
+
+
+def ragged_work(case):
+    pairs = 0
+    for s in range(case.num_spans):
+        lq = int(case.cu_q[s + 1] - case.cu_q[s])
+        lk = int(case.cu_kv[s + 1] - case.cu_kv[s])
+        if case.block_size > 0:
+            i = np.arange(lq, dtype=np.int64)
+            pairs += int(np.minimum(lk, (i // case.block_size + 1) * case.block_size).sum())
+        else:
+            pairs += lq * lk
+    flops = 4 * case.head_dim * case.num_qo_heads * pairs
+    kv_bytes = int(case.cu_kv[-1]) * case.num_kv_heads * case.head_dim * 2 * 2
+    qo_bytes = int(case.cu_q[-1]) * case.num_qo_heads * case.head_dim * 2 * 2
+    return flops, kv_bytes + qo_bytes, kv_bytes
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "tflops": float(p["bf16_tflops"]),
+                "tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "tflops": FALLBACK_TFLOPS,
+                "tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def load_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            entries = json.load(f)
+    except Exception:
+        return None
+    import hashlib
+    for e in entries:
+        if e.get("kernel") != kernel or e.get("workload") != workload:
+            continue
+        src = os.path.join(ROOT, e["source"])
+        try:
+            with open(src, "rb") as f:
+                sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        except Exception:
+            return None
+        if sha == e.get("source_sha"):
+            return float(e["dram_bytes_per_launch"])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.15)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for name, flag in zip(names, r[5:9]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------- our arm
+
+def flush_l2(buf):
+    buf.zero_()
+
+
+def time_layer_calls(ctx, calls, warmup, reps, flush_buf):
+    """Kernel time (attention + merge, ms) per call: CUDA events recorded by the library
+    around its kernels on the launching stream, L2 flushed before every call."""
+    import torch
+    for _ in range(warmup):
+        calls()
+    torch.cuda.synchronize()
+    ctx.enable_kernel_timing(reps)
+    for _ in range(reps):
+        flush_l2(flush_buf)
+        calls()
+    torch.cuda.synchronize()
+    attn, merge = ctx.read_kernel_timing()
+    ctx.enable_kernel_timing(0)
+    return [a + m for a, m in zip(attn, merge)], attn, merge
+
+
+def workload_table(dev, peaks, flush_buf):
+    """Per-layer-call numbers of the five workloads (each one layer, L2 flushed)."""
+    import torch
+    from ragged_attention_encoder_b200 import Context, inputs
+    rows = {}
+    for i in (1, 2, 3, 4, 5):
+        case = inputs.workload(i)
+        paged = hasattr(case, "kv_page_indices")
+        if paged:
+            ctx = Context(case.num_qo_heads, case.num_kv_heads, case.head_dim, case.page_size,
+                          device=dev)
+            kp = inputs.nan_pool(case.num_pages, case.num_kv_heads, case.page_size, case.head_dim, dev)
+            vp = inputs.nan_pool(case.num_pages, case.num_kv_heads, case.page_size, case.head_dim, dev)
+            ctx.write_context(case.k_ctx.to(dev), case.v_ctx.to(dev), case.cu_enc,
+                              case.kv_page_indptr, case.kv_page_indices, kp, vp)
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            plan = ctx.plan_paged(case.qo_indptr, case.kv_page_indptr, case.kv_page_indices,
+                                  case.kv_len, case.num_pages)
+            plan_us = (time.perf_counter() - t0) * 1e6
+            q = case.q.to(dev)
+            out = torch.empty_like(q)
+            call = lambda: ctx.run_paged(plan, q, kp, vp, out)  # noqa: E731
+            flops, nbytes, kvb = paged_work(case)
+        else:
+            ctx = Context(case.num_qo_heads, case.num_kv_heads, case.head_dim, 16, device=dev)
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            plan = ctx.plan_ragged(case.cu_q, None, case.block_size)
+            plan_us = (time.perf_counter() - t0) * 1e6
+            q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+            out = torch.empty_like(q)
+            call = lambda: ctx.run_ragged(plan, q, k, v, out)  # noqa: E731
+            flops, nbytes, kvb = ragged_work(case)
+        tot, attn, merge = time_layer_calls(ctx, call, 3, 20, flush_buf)
+        ctx.check_device_status()
+        t = statistics.median(tot) * 1e-3
+        ta = statistics.median(attn) * 1e-3
+        tc = flops / t / 1e12
+        gbs = nbytes / t / 1e9
+        t_star_spec = max(flops / (SPEC_TC_TFLOPS * 1e12), nbytes / (SPEC_HBM_GBS * 1e9))
+        t_star_meas = max(flops / (peaks["tflops"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
+        bound = "tensor" if flops / (SPEC_TC_TFLOPS * 1e12) > nbytes / (SPEC_HBM_GBS * 1e9) else "hbm"
+        rows[case.name] = {
+            "us_per_layer_call": round(t * 1e6, 2),
+            "attention_kernel_us": round(ta * 1e6, 2),
+            "merge_us": round(statistics.median(merge) * 1e3, 2),
+            "tflops": round(tc, 2),
+            "hbm_gbs": round(gbs, 1),
+            "bound": bound,
+            "roofline_frac_of_spec": round(t_star_spec / t, 4),
+            "roofline_frac_of_measured": round(t_star_meas / t, 4),
+            "tc_frac_of_spec": round(tc / SPEC_TC_TFLOPS, 4),
+            "hbm_frac_of_spec": round(gbs / SPEC_HBM_GBS, 4),
+            "algorithmic_flops": flops,
+            "algorithmic_bytes": nbytes,
+            "tiles": plan.num_tiles,
+            "ctas": plan.num_ctas,
+            "merge_rows": plan.num_merge_rows,
+            "plan_host_us": round(plan_us, 1),
+        }
+        del ctx
+        torch.cuda.empty_cache()
+    return rows
+
+
+def cpu_oracle_rate(case, budget_s):
+    """The float64 oracle on the host cores, repeated over the workload's requests for about
+    budget_s seconds; returns (GB/s of the same algorithmic bytes, seconds, requests)."""
+    import oracle
+    from ragged_attention_encoder_b200 import inputs
+    kp = inputs.nan_pool(case.num_pages, case.num_kv_heads, case.page_size, case.head_dim)
+    vp = inputs.nan_pool(case.num_pages, case.num_kv_heads, case.page_size, case.head_dim)
+    kp, vp = oracle.context_write(case.k_ctx, case.v_ctx, case.cu_enc, case.kv_page_indptr,
+                                  case.kv_page_indices, kp, vp)
+    _, nbytes, _ = paged_work(case)
+    per_req = nbytes / case.batch
+    done, t0 = 0, time.perf_counter()
+    b = 0
+    while True:
+        qo = case.qo_indptr
+        sub_q = case.q[qo[b]:qo[b + 1]]
+        oracle.paged_cross_attention(sub_q, kp, vp, np.array([0, qo[b + 1] - qo[b]]),
+                                     case.kv_page_indptr[b:b + 2] - case.kv_page_indptr[b],
+                                     case.kv_page_indices[case.kv_page_indptr[b]:],
+                                     case.kv_len[b:b + 1])
+        done += 1
+        b = (b + 1) % case.batch
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return per_req * done / el / 1e9, el, done
+
+
+def cpu_cores():
+    try:
+        n = len(os.sched_getaffinity(0))
+    except Exception:
+        n = os.cpu_count() or 1
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        blas = None
+    return n, blas
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from ragged_attention_encoder_b200 import Context, inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    peaks = load_peaks()
+
+    case = inputs.workload(2)
+    flops, nbytes, kv_bytes = paged_work(case)
+    ctx = Context(case.num_qo_heads, case.num_kv_heads, case.head_dim, case.page_size, device=dev)
+
+    # Layer 0 gets the seeded context through the library's context write (timed as a1);
+    # layers 1..31 get seeded random pools drawn on the device.
+    k_pools, v_pools, qs, outs = [], [], [], []
+    kp = inputs.nan_pool(case.num_pages, case.num_kv_heads, case.page_size, case.head_dim, dev)
+    vp = inputs.nan_pool(case.num_pages, case.num_kv_heads, case.page_size, case.head_dim, dev)
+    k_src, v_src = case.k_ctx.to(dev), case.v_ctx.to(dev)
+    ctx.write_context(k_src, v_src, case.cu_enc, case.kv_page_indptr, case.kv_page_indices, kp, vp)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    wtimes = []
+    for _ in range(5):
+        e0.record()
+        ctx.write_context(k_src, v_src, case.cu_enc, case.kv_page_indptr, case.kv_page_indices, kp, vp)
+        e1.record()
+        torch.cuda.synchronize()
+        wtimes.append(e0.elapsed_time(e1))
+    write_bytes = 2 * 2 * int(case.cu_enc[-1]) * case.num_kv_heads * case.head_dim * 2
+    write_ms = statistics.median(wtimes)
+    del k_src, v_src
+    k_pools.append(kp)
+    v_pools.append(vp)
+    qs.append(case.q.to(dev))
+    gen = torch.Generator(device=dev).manual_seed(1000 + rank)
+    shape = (case.num_pages, case.num_kv_heads, case.page_size, case.head_dim)
+    for _ in range(1, LAYERS):
+        k_pools.append(torch.randn(shape, generator=gen, device=dev, dtype=torch.bfloat16))
+        v_pools.append(torch.randn(shape, generator=gen, device=dev, dtype=torch.bfloat16))
+        qs.append(torch.randn(case.q.shape, generator=gen, device=dev, dtype=torch.bfloat16))
+    outs = [torch.empty_like(q) for q in qs]
+
+    def step():
+        plan = ctx.plan_paged(case.qo_indptr, case.kv_page_indptr, case.kv_page_indices,
+                              case.kv_len, case.num_pages)
+        for layer in range(LAYERS):
+            ctx.run_paged(plan, qs[layer], k_pools[layer], v_pools[layer], outs[layer])
+        return plan
+
+    plan = step()
+    for _ in range(max(args.warmup - 1, 0)):
+        step()
+    torch.cuda.synchronize()
+    ctx.check_device_status()
+
+    # ---------------------------------------------------------------- timed region
+    sampler = ClockSampler(local)
+    sampler.start()
+    ctx.enable_kernel_timing(args.steps * LAYERS)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for _ in range(args.steps):
+        step()
+    t_end.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    dev_ms = t_start.elapsed_time(t_end)
+    attn_ms, merge_ms = ctx.read_kernel_timing()
+    ctx.enable_kernel_timing(0)
+    ctx.check_device_status()
+    if world > 1:
+        t = torch.tensor([dev_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dev_ms = float(t.item())
+    ms_per_step = dev_ms / args.steps
+    step_bytes = nbytes * LAYERS
+    value = step_bytes * world / (ms_per_step * 1e-3) / 1e9
+
+    # ---------------------------------------------------------------- end to end
+    q_host = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for q in qs]
+    for h, q in zip(q_host, qs):
+        h.copy_(q)
+    o_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    e2e_steps = max(1, min(args.steps, 50))
+
+    def e2e_step():
+        p = ctx.plan_paged(case.qo_indptr, case.kv_page_indptr, case.kv_page_indices,
+                           case.kv_len, case.num_pages)
+        for layer in range(LAYERS):
+            qs[layer].copy_(q_host[layer], non_blocking=True)
+            ctx.run_paged(p, qs[layer], k_pools[layer], v_pools[layer], outs[layer])
+            o_host[layer].copy_(outs[layer], non_blocking=True)
+        return p
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_start.record()
+    for _ in range(e2e_steps):
+        p = e2e_step()
+    t_end.record()
+    torch.cuda.synchronize()
+    e2e_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = step_bytes * world / (e2e_ms / e2e_steps * 1e-3) / 1e9
+    h2d = sum(q.numel() * 2 for q in qs) + p.raw.image_words * 4
+    d2h = sum(o.numel() * 2 for o in outs)
+
+    # ---------------------------------------------------------------- roofline (decode kernel)
+    attn_mean_ms = statistics.fmean(attn_ms) if attn_ms else float("nan")
+    launch_bytes = nbytes                        # one layer call's algorithmic bytes
+    achieved = launch_bytes / (attn_mean_ms * 1e-3) / 1e9
+    traffic = load_traffic("decode_simt_kernel", "whisper_large_decode")
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic, "kernel": "decode_simt_kernel<64,1>",
+                "peak_source": peaks["source"],
+                "frac_of_spec_8TBs": round(achieved / SPEC_HBM_GBS, 4)}
+
+    result = {
+        "metric": "KV HBM GB/s per B200 (Whisper-large decode cross-attention step: plan + 32 layer calls)",
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; layer 0 from the CPU generator, layers 1-31 device-seeded)",
+        "config": {"workload": "whisper_large_decode", "requests": 64, "q_tokens_per_request": 1,
+                   "context_tokens": 1500, "num_qo_heads": 20, "num_kv_heads": 20,
+                   "head_dim": 64, "page_size": 16, "pool_pages": 16384,
+                   "layers_per_step": LAYERS, "l2": "inputs larger than L2 (491.5 MB K/V per layer)",
+                   "parallelism": f"replicas x{world}"},
+        "us_per_layer_call": round(ms_per_step * 1e3 / LAYERS, 2),
+        "attention_kernel_us": round(attn_mean_ms * 1e3, 2),
+        "merge_kernel_us": round(statistics.fmean(merge_ms) * 1e3, 2) if merge_ms else 0.0,
+        "tflops": round(flops * LAYERS * world / (ms_per_step * 1e-3) / 1e12, 3),
+        "roofline": roofline,
+        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_ms / e2e_steps, 4)},
+        "gpu_launches": int(len(attn_ms) + sum(1 for m in merge_ms if m > 0)),
+        "clocks": clocks,
+        "plan": {"tiles": plan.num_tiles, "ctas": plan.num_ctas, "merge_rows": plan.num_merge_rows},
+        "context_write": {"gbs": round(write_bytes / (write_ms * 1e-3) / 1e9, 1),
+                          "ms": round(write_ms, 4), "bytes": write_bytes},
+    }
+
+    if world == 1 and rank == 0:
+        gbs, secs, reqs = cpu_oracle_rate(case, args.cpu_seconds)
+        cores, blas = cpu_cores()
+        result["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                                  "blas_threads": blas, "kind": "oracle",
+                                  "sample": f"float64 oracle over {reqs} request-layer calls of "
+                                            f"the workload ({secs:.1f} s)"}
+    del k_pools, v_pools
+    torch.cuda.empty_cache()
+    if world == 1 and not args.skip_workloads:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        result["workloads"] = workload_table(dev, peaks, flush)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from ragged_attention_encoder_b200 import inputs
+    import oracle
+    case = inputs.workload(2)
+    _, nbytes, _ = paged_work(case)
+    per_req = nbytes / case.batch
+    kp = inputs.nan_pool(case.num_pages, case.num_kv_heads, case.page_size, case.head_dim)
+    vp = inputs.nan_pool(case.num_pages, case.num_kv_heads, case.page_size, case.head_dim)
+    kp, vp = oracle.context_write(case.k_ctx, case.v_ctx, case.cu_enc, case.kv_page_indptr,
+                                  case.kv_page_indices, kp, vp)
+
+    def one(b):   # one request of one layer call: the bounded sample of a step
+        qo = case.qo_indptr
+        oracle.paged_cross_attention(case.q[qo[b]:qo[b + 1]], kp, vp, np.array([0, 1]),
+                                     case.kv_page_indptr[b:b + 2] - case.kv_page_indptr[b],
+                                     case.kv_page_indices[case.kv_page_indptr[b]:],
+                                     case.kv_len[b:b + 1])
+
+    for w in range(args.warmup):
+        one(w % case.batch)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        one(s % case.batch)
+    el = time.perf_counter() - t0
+    value = per_req * args.steps / el / 1e9
+    cores, blas = cpu_cores()
+    ms = el / args.steps * 1e3
+    print(json.dumps({
+        "impl": "reference",
+        "metric": "KV HBM GB/s per B200 (Whisper-large decode cross-attention step: plan + 32 layer calls)",
+        "value": round(value, 5), "unit": "GB/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": "whisper_large_decode", "requests": 64, "q_tokens_per_request": 1,
+                   "context_tokens": 1500, "num_qo_heads": 20, "num_kv_heads": 20, "head_dim": 64,
+                   "page_size": 16, "pool_pages": 16384, "layers_per_step": LAYERS,
+                   "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": cores,
+                         "blas_threads": blas, "kind": "oracle",
+                         "sample": "each step: the float64 oracle on one request of one layer call"},
+        "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

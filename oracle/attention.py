@@ -136,11 +136,15 @@ def block_causal_key_limit(length: int, block_size: int) -> np.ndarray:
 
 def gather_paged_kv(pool, page_indptr, page_indices, request: int, kv_len: int) -> np.ndarray:
     """Logical K (or V) rows [kv_len, Hkv, d] of one request, read through its page list."""
-    pool = as_f64(pool)
     page_size = pool.shape[2]
     pages = np.asarray(page_indices)[int(page_indptr[request]):int(page_indptr[request + 1])]
     t = np.arange(int(kv_len))
-    return pool[pages[t // page_size], :, t % page_size, :]
+    page_of, slot_of = pages[t // page_size], t % page_size
+    if isinstance(pool, torch.Tensor):   # gather the bf16 rows, then upcast only those
+        rows = pool[torch.from_numpy(page_of.astype(np.int64)), :,
+                    torch.from_numpy(slot_of.astype(np.int64)), :]
+        return as_f64(rows)
+    return as_f64(pool)[page_of, :, slot_of, :]
 
 
 def context_write(k_src: torch.Tensor, v_src: torch.Tensor, cu_enc, page_indptr, page_indices,

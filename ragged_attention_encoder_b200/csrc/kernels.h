@@ -1,0 +1,55 @@
+// Launch interfaces of the CUDA kernels (internal to the library).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "plan.h"
+#include "rae_internal.h"
+
+namespace rae {
+
+// Per-launch view of a plan image that sits in device memory.
+struct DevPlan {
+  const int32_t* cta_ptr;   // [num_ctas + 1]
+  const Tile* tiles;        // [num_tiles]
+  const MergeRow* merge;    // [num_merge]
+  const int32_t* a;         // paged: qo_indptr   ragged: cu_q
+  const int32_t* b;         // paged: kv_len      ragged: cu_kv
+  const int32_t* c;         // paged: kv_page_indptr
+  const int32_t* d;         // paged: kv_page_indices
+  int32_t num_ctas;
+  int32_t num_merge;
+  int32_t block_size;
+};
+
+struct Geometry {
+  int32_t hq, hkv, g, d, page_size;
+};
+
+// Context write: one CTA per page copy.
+cudaError_t launch_context_write(const WriteItem* items, int64_t num_items, const void* k_src,
+                                 const void* v_src, void* k_pool, void* v_pool,
+                                 const Geometry& geo, cudaStream_t stream);
+
+// Paged decode (<= 8 query rows per unit) on CUDA cores.
+cudaError_t launch_decode_simt(const DevPlan& plan, const Geometry& geo, const void* q,
+                               const void* k_pool, const void* v_pool, void* out,
+                               float* part_o, float* part_lse, int* err, float scale_log2,
+                               int64_t timeout_ns, int rows_max, cudaStream_t stream);
+
+// tcgen05 attention over 128-row query tiles (paged or ragged K/V).
+struct TcTensors {
+  CUtensorMap q;   // 3D {d, Hq, total_q}, box {64, g, 128/g}
+  CUtensorMap k;   // paged: 2D {d, pages*Hkv*P}, box {64, P}; ragged: 3D {d, Hkv, T}, box {64,1,128}
+  CUtensorMap v;
+};
+cudaError_t launch_attn_tc(const DevPlan& plan, const Geometry& geo, bool paged,
+                           const TcTensors& maps, void* out, float* part_o, float* part_lse,
+                           int* err, float scale_log2, int64_t timeout_ns, cudaStream_t stream);
+
+// Split-KV merge of partial rows into bf16 outputs.
+cudaError_t launch_merge(const DevPlan& plan, const Geometry& geo, const float* part_o,
+                         const float* part_lse, void* out, cudaStream_t stream);
+
+}  // namespace rae

@@ -1,0 +1,503 @@
+// Host-side plan builder (see plan.h).
+//
+// The plan is the host half of the pages' plan/run split (M* page
+// "mstar.engine.resources.attn.cross", FlashInferCrossManager.plan): it is computed once per
+// step and plan label and then read by every layer's run.  It turns the query packing
+// (QueryPacking.qo_indptr) and the context page table into
+//   * work units: (request, KV head, chunk of query tokens) whose rows are the g = Hq/Hkv
+//     query heads of each token, so one KV head's keys are read once for its whole group;
+//   * a split-KV schedule that gives every CTA of a persistent grid the same number of key
+//     blocks (a unit that straddles two CTAs becomes two or more splits);
+//   * the merge map of the split units.
+#include "plan.h"
+
+#include <algorithm>
+#include <cstring>
+#include <functional>
+#include <queue>
+#include <utility>
+#include <vector>
+
+namespace rae {
+namespace {
+
+int fail(std::string* err, int code, const std::string& msg) {
+  if (err) *err = msg;
+  return code;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t align4(int64_t w) { return (w + 3) & ~int64_t(3); }
+
+struct Unit {
+  int32_t req, kvh, q0, qn, nkeys, rows;
+};
+
+struct Piece {
+  int32_t unit, blk0, nblk, cta;
+};
+
+// Grid capacity (CTAs resident at once) of a kernel family: the decode kernel fits two CTAs
+// per SM; a tcgen05 CTA takes most of an SM's shared memory, so one.
+int32_t grid_for(const rae_config& cfg, int32_t kind) {
+  if (kind == kKindDecodeSimt) return cfg.num_sms * 2;
+  return cfg.num_sms;
+}
+
+// Upper bound of the image size for cfg (words): header, CTA pointers, tiles, merge rows
+// and the request arrays, each 16-byte aligned.
+int64_t max_merge_rows(const rae_config& cfg) {
+  return std::min<int64_t>(cfg.max_partial_rows, int64_t(cfg.max_q_tokens) * cfg.num_qo_heads);
+}
+
+int64_t image_bound(const rae_config& cfg) {
+  int64_t w = kHdrWords;
+  w = align4(w + max_ctas_for(cfg) + 1);
+  w = align4(w + int64_t(cfg.max_tiles) * 8);
+  w = align4(w + max_merge_rows(cfg) * 4);
+  w = align4(w + cfg.max_batch + 1) + align4(cfg.max_batch + 1) + align4(cfg.max_batch + 1);
+  w = align4(w + cfg.max_kv_pages);
+  return w;
+}
+
+// The schedule of one plan, before it is packed into an image.
+struct Schedule {
+  int32_t kind = kKindNone;
+  std::vector<int32_t> cta_ptr;
+  std::vector<Tile> tiles;
+  std::vector<MergeRow> merge;
+};
+
+// Packs a schedule and the request arrays into `image` (compact, offsets in the header).
+int emit_image(const Schedule& sc, const int32_t* a, int64_t na, const int32_t* b, int64_t nb,
+               const int32_t* c, int64_t nc, const int32_t* d, int64_t nd, int32_t* image,
+               int64_t image_words, rae_plan* out, std::string* err) {
+  int64_t w = kHdrWords;
+  const int64_t o_cta = w;
+  w = align4(w + int64_t(sc.cta_ptr.size()));
+  const int64_t o_tiles = w;
+  w = align4(w + int64_t(sc.tiles.size()) * 8);
+  const int64_t o_merge = w;
+  w = align4(w + int64_t(sc.merge.size()) * 4);
+  const int64_t o_a = w;
+  w = align4(w + na);
+  const int64_t o_b = w;
+  w = align4(w + nb);
+  const int64_t o_c = w;
+  w = align4(w + nc);
+  const int64_t o_d = w;
+  w = align4(w + nd);
+  if (w > image_words) return fail(err, RAE_ERR_CAPACITY, "plan image exceeds its slot");
+  std::memset(image, 0, size_t(w) * sizeof(int32_t));
+  if (!sc.cta_ptr.empty()) std::memcpy(image + o_cta, sc.cta_ptr.data(), sc.cta_ptr.size() * 4);
+  if (!sc.tiles.empty()) std::memcpy(image + o_tiles, sc.tiles.data(), sc.tiles.size() * 32);
+  if (!sc.merge.empty()) std::memcpy(image + o_merge, sc.merge.data(), sc.merge.size() * 16);
+  if (na) std::memcpy(image + o_a, a, size_t(na) * 4);
+  if (nb) std::memcpy(image + o_b, b, size_t(nb) * 4);
+  if (nc) std::memcpy(image + o_c, c, size_t(nc) * 4);
+  if (nd) std::memcpy(image + o_d, d, size_t(nd) * 4);
+  image[kHdrMagic] = kPlanMagic;
+  image[kHdrKind] = sc.kind;
+  image[kHdrNumTiles] = int32_t(sc.tiles.size());
+  image[kHdrNumCtas] = int32_t(sc.cta_ptr.empty() ? 0 : sc.cta_ptr.size() - 1);
+  image[kHdrNumMerge] = int32_t(sc.merge.size());
+  image[kHdrOffCtaPtr] = int32_t(o_cta);
+  image[kHdrOffTiles] = int32_t(o_tiles);
+  image[kHdrOffMerge] = int32_t(o_merge);
+  image[kHdrOffA] = int32_t(o_a);
+  image[kHdrOffB] = int32_t(o_b);
+  image[kHdrOffC] = int32_t(o_c);
+  image[kHdrOffD] = int32_t(o_d);
+  out->kind = sc.kind;
+  out->num_tiles = image[kHdrNumTiles];
+  out->num_ctas = image[kHdrNumCtas];
+  out->num_merge_rows = image[kHdrNumMerge];
+  out->image_words = int32_t(w);
+  out->off_cta_ptr = int32_t(o_cta);
+  out->off_tiles = int32_t(o_tiles);
+  out->off_merge = int32_t(o_merge);
+  out->off_a = int32_t(o_a);
+  out->off_b = int32_t(o_b);
+  out->off_c = int32_t(o_c);
+  out->off_d = int32_t(o_d);
+  return RAE_OK;
+}
+
+// Schedules units over the grid: tiles, CTA pointers and merge rows.
+//   blk: keys per block; ovh: per-tile overhead in blocks; g: query heads per KV head.
+//   lpt_factor: whole units are scheduled longest-first when every CTA's share is at least
+//   lpt_factor times the largest unit; otherwise the balanced contiguous partition is used.
+int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units, int32_t blk,
+             int32_t ovh, int32_t g, int32_t lpt_factor, Schedule* sc, std::string* err) {
+  const int32_t grid = grid_for(cfg, kind);
+  const int64_t nu = int64_t(units.size());
+  std::vector<int64_t> nb(nu), cost(nu);
+  int64_t total = 0, maxc = 0;
+  for (int64_t u = 0; u < nu; ++u) {
+    nb[u] = ceil_div(units[u].nkeys, blk);
+    cost[u] = nb[u] + ovh;
+    total += cost[u];
+    maxc = std::max(maxc, cost[u]);
+  }
+
+  std::vector<Piece> pieces;
+  std::vector<int32_t> npieces(nu, 0);
+  int32_t num_ctas = 0;
+
+  auto lpt = [&]() {
+    // Longest-processing-time-first: whole units, each to the least-loaded CTA.
+    pieces.clear();
+    std::fill(npieces.begin(), npieces.end(), 0);
+    std::vector<int64_t> order(nu);
+    for (int64_t u = 0; u < nu; ++u) order[u] = u;
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int64_t a, int64_t b) { return cost[a] > cost[b]; });
+    const int32_t ctas = int32_t(std::min<int64_t>(grid, nu));
+    using Load = std::pair<int64_t, int32_t>;
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+    for (int32_t c = 0; c < ctas; ++c) heap.push({0, c});
+    for (int64_t u : order) {
+      Load l = heap.top();
+      heap.pop();
+      pieces.push_back({int32_t(u), 0, int32_t(nb[u]), l.second});
+      npieces[u] = 1;
+      heap.push({l.first + cost[u], l.second});
+    }
+    std::stable_sort(pieces.begin(), pieces.end(),
+                     [](const Piece& a, const Piece& b) { return a.cta < b.cta; });
+    num_ctas = ctas;
+  };
+
+  // Greedy fill of CTAs with capacity q (blocks + overhead per piece), in unit order;
+  // returns the CTAs used, and the pieces when `emit` is set.
+  auto greedy = [&](int64_t q, bool emit) -> int64_t {
+    int64_t c = 0, cap = q;
+    bool used = false;
+    for (int64_t u = 0; u < nu; ++u) {
+      int64_t rb = nb[u], s = 0;
+      do {
+        if (used && cap <= ovh) {
+          ++c;
+          cap = q;
+          used = false;
+        }
+        const int64_t take = std::min<int64_t>(rb, std::max<int64_t>(cap - ovh, 1));
+        if (emit) {
+          pieces.push_back({int32_t(u), int32_t(s), int32_t(take), int32_t(c)});
+          npieces[u] += 1;
+        }
+        used = true;
+        cap -= take + ovh;
+        s += take;
+        rb -= take;
+      } while (rb > 0);
+    }
+    return c + 1;
+  };
+
+  auto contiguous = [&]() {
+    // Every CTA takes an equal share of the blocks of all units laid end to end; a unit cut
+    // by a CTA boundary becomes several splits, merged afterwards in split order.  The share
+    // is the smallest capacity whose greedy fill needs no more CTAs than the grid holds.
+    pieces.clear();
+    std::fill(npieces.begin(), npieces.end(), 0);
+    int64_t lo = std::max<int64_t>(ceil_div(total, grid), ovh + 1);
+    int64_t hi = lo;
+    while (greedy(hi, false) > grid) hi *= 2;
+    while (lo < hi) {
+      const int64_t mid = lo + (hi - lo) / 2;
+      if (greedy(mid, false) <= grid) hi = mid; else lo = mid + 1;
+    }
+    num_ctas = int32_t(greedy(lo, true));
+  };
+
+  if (nu == 0) {
+    num_ctas = 0;
+  } else if (maxc * lpt_factor <= total / grid) {
+    lpt();   // many small units: whole units balance well, no merge needed
+  } else {
+    contiguous();
+    int64_t prow = 0;
+    for (int64_t u = 0; u < nu; ++u)
+      if (npieces[u] > 1) prow += int64_t(npieces[u]) * units[u].rows;
+    if (prow > cfg.max_partial_rows || prow > max_merge_rows(cfg)) lpt();
+  }
+
+  if (int64_t(pieces.size()) > cfg.max_tiles)
+    return fail(err, RAE_ERR_CAPACITY,
+                "plan needs " + std::to_string(pieces.size()) + " tiles > max_tiles " +
+                    std::to_string(cfg.max_tiles));
+
+  // Partial rows of the split units, and the merge map.
+  std::vector<int64_t> part_base(nu, -1);
+  int64_t prow = 0, nmerge = 0;
+  for (int64_t u = 0; u < nu; ++u) {
+    if (npieces[u] > 1) {
+      part_base[u] = prow;
+      prow += int64_t(npieces[u]) * units[u].rows;
+      nmerge += units[u].rows;
+    }
+  }
+  if (prow > cfg.max_partial_rows || nmerge > max_merge_rows(cfg))
+    return fail(err, RAE_ERR_CAPACITY, "split-KV partials exceed max_partial_rows");
+
+  sc->kind = kind;
+  sc->cta_ptr.assign(size_t(num_ctas) + 1, 0);
+  sc->tiles.resize(pieces.size());
+  std::vector<int32_t> seen(nu, 0);
+  int32_t cur = -1;
+  for (size_t i = 0; i < pieces.size(); ++i) {
+    const Piece& p = pieces[i];
+    while (cur < p.cta) sc->cta_ptr[size_t(++cur)] = int32_t(i);
+    const Unit& un = units[size_t(p.unit)];
+    Tile t;
+    t.req = un.req;
+    t.kv_head = un.kvh;
+    t.q0 = un.q0;
+    t.qn = un.qn;
+    t.kv0 = int32_t(std::min<int64_t>(int64_t(p.blk0) * blk, un.nkeys));
+    t.kv1 = int32_t(std::min<int64_t>(int64_t(p.blk0 + p.nblk) * blk, un.nkeys));
+    t.split = seen[size_t(p.unit)]++;
+    t.part = part_base[size_t(p.unit)] < 0
+                 ? -1
+                 : int32_t(part_base[size_t(p.unit)] + int64_t(t.split) * un.rows);
+    sc->tiles[i] = t;
+  }
+  while (cur < num_ctas) sc->cta_ptr[size_t(++cur)] = int32_t(pieces.size());
+
+  sc->merge.clear();
+  sc->merge.reserve(size_t(nmerge));
+  for (int64_t u = 0; u < nu; ++u) {
+    if (part_base[size_t(u)] < 0) continue;
+    const Unit& un = units[size_t(u)];
+    for (int32_t r = 0; r < un.rows; ++r) {
+      MergeRow mr;
+      const int32_t tok = un.q0 + r / g;
+      const int32_t head = un.kvh * g + r % g;
+      mr.out_row = tok * cfg.num_qo_heads + head;
+      mr.nsplit = npieces[size_t(u)];
+      mr.part0 = int32_t(part_base[size_t(u)] + r);
+      mr.stride = un.rows;
+      sc->merge.push_back(mr);
+    }
+  }
+  return RAE_OK;
+}
+
+int check_indptr(const int32_t* a, int32_t n, const char* name, std::string* err) {
+  if (!a) return fail(err, RAE_ERR_INVALID_ARG, std::string(name) + " is NULL");
+  if (a[0] != 0) return fail(err, RAE_ERR_INVALID_ARG, std::string(name) + "[0] must be 0");
+  for (int32_t i = 0; i < n; ++i)
+    if (a[i + 1] < a[i])
+      return fail(err, RAE_ERR_INVALID_ARG,
+                  std::string(name) + " decreases at " + std::to_string(i));
+  return RAE_OK;
+}
+
+}  // namespace
+
+int check_config(const rae_config& cfg, std::string* err) {
+  if (cfg.head_dim != 64 && cfg.head_dim != 128)
+    return fail(err, RAE_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (cfg.page_size != 16 && cfg.page_size != 32 && cfg.page_size != 64)
+    return fail(err, RAE_ERR_UNSUPPORTED, "page_size must be 16, 32 or 64");
+  if (cfg.num_qo_heads <= 0 || cfg.num_kv_heads <= 0)
+    return fail(err, RAE_ERR_INVALID_ARG, "head counts must be positive");
+  if (cfg.num_qo_heads % cfg.num_kv_heads != 0)
+    return fail(err, RAE_ERR_UNSUPPORTED, "num_qo_heads must be a multiple of num_kv_heads");
+  if (cfg.num_qo_heads / cfg.num_kv_heads > kTcRows)
+    return fail(err, RAE_ERR_UNSUPPORTED, "more than 128 query heads per KV head");
+  if (cfg.max_batch < 1 || cfg.max_q_tokens < 1 || cfg.max_kv_pages < 1 || cfg.max_tiles < 1 ||
+      cfg.max_partial_rows < 0)
+    return fail(err, RAE_ERR_INVALID_ARG, "capacities must be positive");
+  if (cfg.num_sms <= 0) return fail(err, RAE_ERR_INVALID_ARG, "num_sms must be positive");
+  if (int64_t(cfg.max_q_tokens) * cfg.num_qo_heads >= (int64_t(1) << 31))
+    return fail(err, RAE_ERR_CAPACITY, "max_q_tokens * num_qo_heads overflows int32");
+  if (image_bound(cfg) >= (int64_t(1) << 31))
+    return fail(err, RAE_ERR_CAPACITY, "plan image too large");
+  return RAE_OK;
+}
+
+int32_t max_ctas_for(const rae_config& cfg) { return cfg.num_sms * 2; }
+
+int64_t image_words_for(const rae_config& cfg) { return image_bound(cfg); }
+
+int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
+                     const int32_t* kv_page_indptr, const int32_t* kv_page_indices,
+                     const int32_t* kv_len, int32_t batch, int32_t num_pages, int32_t* image,
+                     int64_t image_words, rae_plan* out, std::string* err) {
+  int rc = check_config(cfg, err);
+  if (rc) return rc;
+  if (!image) return fail(err, RAE_ERR_INVALID_ARG, "image is NULL");
+  if (!out) return fail(err, RAE_ERR_INVALID_ARG, "out is NULL");
+  if (batch < 0) return fail(err, RAE_ERR_INVALID_ARG, "batch < 0");
+  if (batch > cfg.max_batch) return fail(err, RAE_ERR_CAPACITY, "batch > max_batch");
+  if ((rc = check_indptr(qo_indptr, batch, "qo_indptr", err))) return rc;
+  if ((rc = check_indptr(kv_page_indptr, batch, "kv_page_indptr", err))) return rc;
+  if (batch > 0 && !kv_len) return fail(err, RAE_ERR_INVALID_ARG, "kv_len is NULL");
+  const int32_t total_q = qo_indptr[batch];
+  const int32_t nnz = kv_page_indptr[batch];
+  if (total_q > cfg.max_q_tokens) return fail(err, RAE_ERR_CAPACITY, "total queries > max_q_tokens");
+  if (nnz > cfg.max_kv_pages) return fail(err, RAE_ERR_CAPACITY, "page entries > max_kv_pages");
+  if (nnz > 0 && !kv_page_indices) return fail(err, RAE_ERR_INVALID_ARG, "kv_page_indices is NULL");
+  if (num_pages < 0) return fail(err, RAE_ERR_INVALID_ARG, "num_pages < 0");
+  if (int64_t(num_pages) * cfg.num_kv_heads * cfg.page_size >= (int64_t(1) << 31))
+    return fail(err, RAE_ERR_CAPACITY, "pool rows overflow int32");
+  for (int32_t i = 0; i < nnz; ++i)
+    if (kv_page_indices[i] < 0 || kv_page_indices[i] >= num_pages)
+      return fail(err, RAE_ERR_INVALID_ARG,
+                  "page id " + std::to_string(kv_page_indices[i]) + " at " + std::to_string(i) +
+                      " outside [0, num_pages)");
+  for (int32_t b = 0; b < batch; ++b) {
+    if (kv_len[b] < 0) return fail(err, RAE_ERR_INVALID_ARG, "kv_len < 0");
+    int64_t need = ceil_div(kv_len[b], cfg.page_size);
+    if (kv_page_indptr[b + 1] - kv_page_indptr[b] < need)
+      return fail(err, RAE_ERR_INVALID_ARG,
+                  "request " + std::to_string(b) + " has fewer pages than kv_len needs");
+  }
+
+  const int32_t g = cfg.num_qo_heads / cfg.num_kv_heads;
+  int32_t max_qlen = 0;
+  for (int32_t b = 0; b < batch; ++b) max_qlen = std::max(max_qlen, qo_indptr[b + 1] - qo_indptr[b]);
+  const bool simt = int64_t(max_qlen) * g <= kSimtMaxRows;
+  const int32_t kind = simt ? kKindDecodeSimt : kKindTcPaged;
+  const int32_t tok_per_unit = simt ? std::max(max_qlen, 1) : kTcRows / g;
+
+  std::vector<Unit> units;
+  for (int32_t b = 0; b < batch; ++b) {
+    const int32_t qlen = qo_indptr[b + 1] - qo_indptr[b];
+    for (int32_t h = 0; h < cfg.num_kv_heads; ++h)
+      for (int32_t t = 0; t < qlen; t += tok_per_unit) {
+        Unit u;
+        u.req = b;
+        u.kvh = h;
+        u.q0 = qo_indptr[b] + t;
+        u.qn = std::min(tok_per_unit, qlen - t);
+        u.nkeys = kv_len[b];
+        u.rows = u.qn * g;
+        units.push_back(u);
+      }
+  }
+
+  out->batch = batch;
+  out->total_q = total_q;
+  out->block_size = 0;
+  int32_t rows_max = 0;
+  for (const Unit& u : units) rows_max = std::max(rows_max, u.rows);
+  out->rows_max = rows_max;
+  Schedule sc;
+  // The decode kernel is HBM bound and short: an even split of the bytes over the grid
+  // matters more than the small merge it costs.
+  rc = simt ? schedule(cfg, kind, units, kSimtChunkKeys, 2, g, 64, &sc, err)
+            : schedule(cfg, kind, units, kTcBlockKeys, 1, g, 4, &sc, err);
+  if (rc) return rc;
+  rc = emit_image(sc, qo_indptr, batch + 1, kv_len, batch, kv_page_indptr, batch + 1,
+                  kv_page_indices, nnz, image, image_words, out, err);
+  if (rc) return rc;
+  image[kHdrBatch] = batch;
+  image[kHdrTotalQ] = total_q;
+  image[kHdrBlockSize] = 0;
+  image[kHdrRowsMax] = rows_max;
+  return RAE_OK;
+}
+
+int build_ragged_plan(const rae_config& cfg, const int32_t* cu_q, const int32_t* cu_kv,
+                      int32_t num_spans, int32_t block_size, int32_t* image, int64_t image_words,
+                      rae_plan* out, std::string* err) {
+  int rc = check_config(cfg, err);
+  if (rc) return rc;
+  if (!image) return fail(err, RAE_ERR_INVALID_ARG, "image is NULL");
+  if (!out) return fail(err, RAE_ERR_INVALID_ARG, "out is NULL");
+  if (num_spans < 0) return fail(err, RAE_ERR_INVALID_ARG, "num_spans < 0");
+  if (num_spans > cfg.max_batch) return fail(err, RAE_ERR_CAPACITY, "num_spans > max_batch");
+  if (block_size < 0) return fail(err, RAE_ERR_INVALID_ARG, "block_size < 0");
+  if ((rc = check_indptr(cu_q, num_spans, "cu_seqlens_q", err))) return rc;
+  const int32_t* kv = cu_kv ? cu_kv : cu_q;
+  if (cu_kv && (rc = check_indptr(cu_kv, num_spans, "cu_seqlens_kv", err))) return rc;
+  const int32_t total_q = cu_q[num_spans];
+  if (total_q > cfg.max_q_tokens) return fail(err, RAE_ERR_CAPACITY, "total queries > max_q_tokens");
+
+  const int32_t g = cfg.num_qo_heads / cfg.num_kv_heads;
+  const int32_t tok_per_unit = kTcRows / g;
+  std::vector<Unit> units;
+  for (int32_t s = 0; s < num_spans; ++s) {
+    const int32_t lq = cu_q[s + 1] - cu_q[s];
+    const int32_t lk = kv[s + 1] - kv[s];
+    for (int32_t h = 0; h < cfg.num_kv_heads; ++h)
+      for (int32_t t = 0; t < lq; t += tok_per_unit) {
+        Unit u;
+        u.req = s;
+        u.kvh = h;
+        u.q0 = cu_q[s] + t;
+        u.qn = std::min(tok_per_unit, lq - t);
+        int64_t lim = lk;
+        if (block_size > 0) {
+          const int64_t last = t + u.qn - 1;  // local position of the chunk's last token
+          lim = std::min<int64_t>(lk, (last / block_size + 1) * int64_t(block_size));
+        }
+        u.nkeys = int32_t(lim);
+        u.rows = u.qn * g;
+        units.push_back(u);
+      }
+  }
+  out->batch = num_spans;
+  out->total_q = total_q;
+  out->block_size = block_size;
+  out->rows_max = 0;
+  for (const Unit& u : units) out->rows_max = std::max(out->rows_max, u.rows);
+  Schedule sc;
+  rc = schedule(cfg, kKindTcRagged, units, kTcBlockKeys, 1, g, 4, &sc, err);
+  if (rc) return rc;
+  rc = emit_image(sc, cu_q, num_spans + 1, kv, num_spans + 1, nullptr, 0, nullptr, 0, image,
+                  image_words, out, err);
+  if (rc) return rc;
+  image[kHdrBatch] = num_spans;
+  image[kHdrTotalQ] = total_q;
+  image[kHdrBlockSize] = block_size;
+  image[kHdrRowsMax] = out->rows_max;
+  return RAE_OK;
+}
+
+int build_write_items(const rae_config& cfg, const int32_t* cu_enc, const int32_t* page_indptr,
+                      const int32_t* page_indices, int32_t batch, int32_t num_pages,
+                      WriteItem* items, int64_t max_items, int64_t* num_items, std::string* err) {
+  int rc = check_config(cfg, err);
+  if (rc) return rc;
+  if (batch < 0) return fail(err, RAE_ERR_INVALID_ARG, "batch < 0");
+  if (batch > cfg.max_batch) return fail(err, RAE_ERR_CAPACITY, "batch > max_batch");
+  if ((rc = check_indptr(cu_enc, batch, "cu_enc", err))) return rc;
+  if ((rc = check_indptr(page_indptr, batch, "page_indptr", err))) return rc;
+  const int32_t nnz = page_indptr[batch];
+  if (nnz > 0 && !page_indices) return fail(err, RAE_ERR_INVALID_ARG, "page_indices is NULL");
+  if (num_pages < 0) return fail(err, RAE_ERR_INVALID_ARG, "num_pages < 0");
+  if (int64_t(num_pages) * cfg.num_kv_heads * cfg.page_size >= (int64_t(1) << 31))
+    return fail(err, RAE_ERR_CAPACITY, "pool rows overflow int32");
+  std::vector<uint8_t> used(size_t(num_pages), 0);
+  int64_t n = 0;
+  for (int32_t b = 0; b < batch; ++b) {
+    const int32_t len = cu_enc[b + 1] - cu_enc[b];
+    const int64_t need = ceil_div(len, cfg.page_size);
+    if (page_indptr[b + 1] - page_indptr[b] < need)
+      return fail(err, RAE_ERR_INVALID_ARG,
+                  "request " + std::to_string(b) + " has fewer pages than its context needs");
+    for (int64_t i = 0; i < need; ++i) {
+      const int32_t page = page_indices[page_indptr[b] + i];
+      if (page < 0 || page >= num_pages)
+        return fail(err, RAE_ERR_INVALID_ARG, "page id " + std::to_string(page) + " out of range");
+      if (used[size_t(page)])
+        return fail(err, RAE_ERR_INVALID_ARG,
+                    "page id " + std::to_string(page) + " written twice in one call");
+      used[size_t(page)] = 1;
+      if (n >= max_items) return fail(err, RAE_ERR_CAPACITY, "write needs more pages than max_kv_pages");
+      WriteItem& it = items[n++];
+      it.src_row = cu_enc[b] + int32_t(i) * cfg.page_size;
+      it.ntok = std::min<int32_t>(cfg.page_size, len - int32_t(i) * cfg.page_size);
+      it.page = page;
+      it.pad = 0;
+    }
+  }
+  *num_items = n;
+  return RAE_OK;
+}
+
+}  // namespace rae

@@ -1,0 +1,72 @@
+// Internal definitions shared by the host plan builder and the CUDA kernels.
+#pragma once
+#include <stdint.h>
+
+namespace rae {
+
+constexpr int32_t kPlanMagic = 0x52414531;  // "RAE1"
+
+// Kernel families chosen by the plan.
+enum Kind : int32_t {
+  kKindNone = 0,
+  kKindDecodeSimt = 1,   // paged, <= 8 query rows per (request, KV head): CUDA cores, HBM bound
+  kKindTcPaged = 2,      // paged, tcgen05 tiles of 128 query rows
+  kKindTcRagged = 3,     // ragged spans, tcgen05 tiles of 128 query rows
+};
+
+// Plan image header (int32 words).
+enum Hdr : int32_t {
+  kHdrMagic = 0,
+  kHdrKind = 1,
+  kHdrNumTiles = 2,
+  kHdrNumCtas = 3,
+  kHdrNumMerge = 4,
+  kHdrBatch = 5,
+  kHdrTotalQ = 6,
+  kHdrBlockSize = 7,
+  kHdrOffCtaPtr = 8,
+  kHdrOffTiles = 9,
+  kHdrOffMerge = 10,
+  kHdrOffA = 11,   // paged: qo_indptr [B+1]        ragged: cu_q [S+1]
+  kHdrOffB = 12,   // paged: kv_len [B]             ragged: cu_kv [S+1]
+  kHdrOffC = 13,   // paged: kv_page_indptr [B+1]   ragged: unused
+  kHdrOffD = 14,   // paged: kv_page_indices [nnz]  ragged: unused
+  kHdrRowsMax = 15,
+  kHdrWords = 16,
+};
+
+// One work tile: query rows of one (request, KV head, query chunk) against a key range.
+// Rows are ordered (token, head-in-group): row = tok * g + j.
+struct Tile {
+  int32_t req;        // request (paged) or span (ragged)
+  int32_t kv_head;
+  int32_t q0;         // first query token (global packed index)
+  int32_t qn;         // query tokens in the tile
+  int32_t kv0;        // first key (logical index within the request's keys)
+  int32_t kv1;        // one past the last key of this tile
+  int32_t part;       // -1: write out directly; else first partial row of this split
+  int32_t split;      // split index within the unit (0 when unsplit)
+};
+static_assert(sizeof(Tile) == 32, "tile is 8 words");
+
+// One output row produced by a split-KV merge.
+struct MergeRow {
+  int32_t out_row;    // token * Hq + head
+  int32_t nsplit;
+  int32_t part0;      // partial row of split 0
+  int32_t stride;     // distance between splits, in partial rows
+};
+static_assert(sizeof(MergeRow) == 16, "merge row is 4 words");
+
+// Work-unit block granularity in keys: the tcgen05 kernels step 128 keys at a time, the
+// SIMT decode kernel 16 keys (one 16-row chunk of a page).
+constexpr int32_t kTcBlockKeys = 128;
+constexpr int32_t kSimtChunkKeys = 16;
+constexpr int32_t kSimtMaxRows = 8;
+constexpr int32_t kTcRows = 128;
+
+// Workspace layout: [error words | slot 0 image | slot 1 image | write staging | partial O |
+// partial lse], every region 256-byte aligned.
+constexpr int64_t kErrWordsBytes = 256;
+
+}  // namespace rae

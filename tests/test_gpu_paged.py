@@ -1,0 +1,199 @@
+"""Paged cross-attention and the context write on the GPU, against the float64 oracle.
+
+Inputs are the seeded workloads of ragged_attention_encoder_b200.inputs; the pools start as
+bf16 NaN so that a stray read of an untouched slot poisons the output.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from ragged_attention_encoder_b200 import Context, inputs
+
+from gpu_util import (assert_close, context_for, gpu_pools, oracle_paged, oracle_pools,
+                      run_paged)
+
+pytestmark = pytest.mark.gpu
+
+
+# ------------------------------------------------------------------------- context write
+
+@pytest.mark.parametrize("wl", [1, 3])
+def test_context_write_is_bit_exact(wl):
+    case = inputs.workload(wl)
+    ctx = context_for(case)
+    kp, vp = gpu_pools(case, ctx)
+    torch.cuda.synchronize()
+    rk, rv = oracle_pools(case)
+    assert torch.equal(kp.cpu().view(torch.int16), rk.view(torch.int16))
+    assert torch.equal(vp.cpu().view(torch.int16), rv.view(torch.int16))
+
+
+def test_context_write_whisper_pool_is_bit_exact():
+    """The full 16384-page pool of the Whisper-large decode workload."""
+    case = inputs.workload(2)
+    ctx = context_for(case)
+    kp, vp = gpu_pools(case, ctx)
+    torch.cuda.synchronize()
+    rk, rv = oracle_pools(case)
+    assert torch.equal(kp.cpu().view(torch.int16), rk.view(torch.int16))
+    assert torch.equal(vp.cpu().view(torch.int16), rv.view(torch.int16))
+
+
+def test_context_write_rejects_duplicate_pages():
+    case = inputs.paged_case(31, q_lens=[1, 1], ctx_lens=[10, 10], num_qo_heads=2, num_kv_heads=1,
+                             head_dim=64, page_size=16, pool_pages=4)
+    ctx = context_for(case)
+    kp = inputs.nan_pool(4, 1, 16, 64, "cuda")
+    vp = inputs.nan_pool(4, 1, 16, 64, "cuda")
+    with pytest.raises(ValueError, match="twice"):
+        ctx.write_context(case.k_ctx.cuda(), case.v_ctx.cuda(), case.cu_enc, [0, 1, 2], [3, 3],
+                          kp, vp)
+    with pytest.raises(ValueError, match="range"):
+        ctx.write_context(case.k_ctx.cuda(), case.v_ctx.cuda(), case.cu_enc, [0, 1, 2], [3, 4],
+                          kp, vp)
+    torch.cuda.synchronize()
+    assert torch.all(kp.view(torch.int16) == inputs.BF16_NAN_BITS)
+
+
+# --------------------------------------------------------------------------- workloads
+
+def test_tiny_paged_decode():
+    case = inputs.workload(1)
+    out, plan, *_ = run_paged(case)
+    assert_close(out, oracle_paged(case), what="tiny")
+
+
+def test_whisper_large_decode():
+    case = inputs.workload(2)
+    out, plan, *_ = run_paged(case)
+    assert plan.num_merge_rows > 0      # the balanced schedule splits some requests
+    assert_close(out, oracle_paged(case), what="whisper")
+
+
+def test_packed_multitoken_cross():
+    case = inputs.workload(3)
+    out, plan, *_ = run_paged(case)
+    assert_close(out, oracle_paged(case), what="multitoken")
+
+
+def test_long_context_splitkv_sampled():
+    """Full-size long-context workload in the benchmark's launch configuration; sampled rows
+    are checked one by one against attention over each request's packed context K/V."""
+    case = inputs.workload(5)
+    out, plan, *_ = run_paged(case)
+    assert plan.num_merge_rows > 0
+    g = case.num_qo_heads // case.num_kv_heads
+    rng = np.random.default_rng(5)
+    o = out.float().cpu().numpy()
+    assert np.all(np.isfinite(o))
+    scale = 1.0 / np.sqrt(case.head_dim)
+    for b in rng.choice(case.batch, 3, replace=False):
+        c0, c1 = case.cu_enc[b], case.cu_enc[b + 1]
+        for kvh in rng.choice(case.num_kv_heads, 2, replace=False):
+            kb = oracle.as_f64(case.k_ctx[c0:c1, kvh])
+            vb = oracle.as_f64(case.v_ctx[c0:c1, kvh])
+            for t in range(case.qo_indptr[b], case.qo_indptr[b + 1]):
+                heads = list(range(kvh * g, kvh * g + g))
+                qrows = oracle.as_f64(case.q[t, heads])
+                ref = oracle.attention_rows(qrows, kb, vb, scale)
+                assert_close(o[t, heads], ref, what=f"req {b} tok {t}")
+
+
+# ---------------------------------------------------------------------------- edge cases
+
+@pytest.mark.parametrize("P", [16, 32, 64])
+@pytest.mark.parametrize("d", [64, 128])
+def test_kv_len_around_page_boundaries(P, d):
+    lens = [1, P - 1, P, P + 1, 2 * P + 3]
+    case = inputs.paged_case(40 + P + d, q_lens=[1, 2, 1, 3, 1], ctx_lens=lens, num_qo_heads=4,
+                             num_kv_heads=2, head_dim=d, page_size=P, pool_pages=64)
+    out, *_ = run_paged(case)
+    assert_close(out, oracle_paged(case), what=f"P={P} d={d}")
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 4), (8, 2), (8, 1), (6, 2), (40, 5)])
+@pytest.mark.parametrize("qmax", [1, 40])
+def test_gqa_groups_and_query_lengths(hq, hkv, qmax):
+    case = inputs.paged_case(50 + hq + hkv + qmax, q_lens=(0, qmax, 6), ctx_lens=(1, 600, 6),
+                             num_qo_heads=hq, num_kv_heads=hkv, head_dim=64, page_size=16)
+    out, plan, *_ = run_paged(case)
+    assert_close(out, oracle_paged(case), what=f"{hq}/{hkv} q<={qmax}")
+
+
+def test_empty_context_gives_zero():
+    case = inputs.paged_case(61, q_lens=[2, 1, 3], ctx_lens=[0, 5, 0], num_qo_heads=4,
+                             num_kv_heads=2, head_dim=64, page_size=16, pool_pages=4)
+    out, *_ = run_paged(case)
+    ref = oracle_paged(case)
+    assert np.all(ref[0:2] == 0) and np.all(ref[3:] == 0)
+    assert_close(out, ref, what="empty ctx")
+    case = inputs.paged_case(62, q_lens=[40, 0, 30], ctx_lens=[0, 5, 700], num_qo_heads=8,
+                             num_kv_heads=2, head_dim=128, page_size=16)
+    out, plan, *_ = run_paged(case)
+    assert plan.kernel_kind == 2
+    assert_close(out, oracle_paged(case), what="empty ctx tc")
+
+
+@pytest.mark.parametrize("num_sms", [1, 2, 5])
+@pytest.mark.parametrize("qmax", [1, 50])
+def test_forced_splits_agree_with_oracle_and_unsplit(num_sms, qmax):
+    case = inputs.paged_case(70 + num_sms + qmax, q_lens=(1, qmax, 3), ctx_lens=(300, 3000, 3),
+                             num_qo_heads=8, num_kv_heads=2, head_dim=128, page_size=32)
+    ref = oracle_paged(case)
+    out_split, plan, *_ = run_paged(case, num_sms=num_sms)
+    assert plan.num_merge_rows > 0
+    assert_close(out_split, ref, what="split")
+    out_full, plan_full, *_ = run_paged(case)
+    assert_close(out_full, ref, what="unsplit")
+
+
+def test_explicit_scale():
+    case = inputs.paged_case(81, q_lens=[3, 20], ctx_lens=[100, 257], num_qo_heads=8,
+                             num_kv_heads=2, head_dim=64, page_size=16)
+    out, *_ = run_paged(case, sm_scale=0.05)
+    assert_close(out, oracle_paged(case, scale=0.05), what="scale")
+
+
+# --------------------------------------------------------------------------- metamorphic
+
+@pytest.mark.parametrize("qmax", [1, 60])
+def test_page_permutation_gives_bit_identical_output(qmax):
+    case = inputs.paged_case(90 + qmax, q_lens=(1, qmax, 4), ctx_lens=(100, 900, 4),
+                             num_qo_heads=8, num_kv_heads=4, head_dim=64, page_size=16)
+    out1, *_ = run_paged(case)
+    perm = np.random.default_rng(1).permutation(case.num_pages).astype(np.int32)
+    case.kv_page_indices = perm[case.kv_page_indices]
+    out2, *_ = run_paged(case)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+@pytest.mark.parametrize("wl", [2, 3])
+def test_repeated_runs_are_bit_identical(wl):
+    case = inputs.workload(wl)
+    out1, plan, ctx, kp, vp = run_paged(case)
+    q = case.q.cuda()
+    out2 = ctx.run_paged(plan, q, kp, vp)
+    torch.cuda.synchronize()
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def test_mha_duplicate_of_gqa_matches_oracle():
+    case = inputs.paged_case(95, q_lens=(1, 30, 3), ctx_lens=(50, 500, 3), num_qo_heads=8,
+                             num_kv_heads=2, head_dim=64, page_size=16)
+    ref = oracle_paged(case)
+    case.k_ctx = case.k_ctx.repeat_interleave(4, dim=1).contiguous()
+    case.v_ctx = case.v_ctx.repeat_interleave(4, dim=1).contiguous()
+    case.num_kv_heads = 8
+    out, *_ = run_paged(case)
+    assert_close(out, ref, what="mha")
+
+
+def test_constant_v_returns_v():
+    case = inputs.paged_case(96, q_lens=(1, 50, 4), ctx_lens=(10, 800, 4), num_qo_heads=8,
+                             num_kv_heads=2, head_dim=128, page_size=16)
+    c = torch.randn(case.head_dim).to(torch.bfloat16)
+    case.v_ctx = c.expand_as(case.v_ctx).contiguous()
+    out, *_ = run_paged(case)
+    o = out.float().cpu()
+    assert torch.equal(o, c.float().expand_as(o)), float((o - c.float()).abs().max())

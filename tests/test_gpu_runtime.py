@@ -1,0 +1,83 @@
+"""Runtime behaviour on the GPU: plan slots, staging race, stale plans and status words."""
+import numpy as np
+import pytest
+import torch
+
+from ragged_attention_encoder_b200 import Context, inputs
+
+from gpu_util import assert_close, gpu_pools, oracle_paged
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(seed, qmax=1):
+    return inputs.paged_case(seed, q_lens=(1, qmax, 5), ctx_lens=(20, 400, 5), num_qo_heads=8,
+                             num_kv_heads=2, head_dim=64, page_size=16, pool_pages=200)
+
+
+def test_double_buffered_plans_under_a_busy_stream():
+    """plan(N+1) and plan(N+2) are issued while run(N) still waits behind a long kernel on the
+    stream; every run must still see its own plan (the staging race of the cross manager)."""
+    cases = [_case(200), _case(201, qmax=3), _case(202)]
+    span = 130                      # pages reserved per case (5 requests x <= 25 pages)
+    num_pages = span * len(cases)
+    ctx = Context(8, 2, 64, 16)
+    k_pool = inputs.nan_pool(num_pages, 2, 16, 64, "cuda")
+    v_pool = inputs.nan_pool(num_pages, 2, 16, 64, "cuda")
+    outs = []
+    torch.cuda._sleep(200_000_000)   # keep the stream busy for a while
+    for i, c in enumerate(cases):
+        c.kv_page_indices = np.arange(c.kv_page_indices.size, dtype=np.int32) + span * i
+        c.num_pages = num_pages
+        ctx.write_context(c.k_ctx.cuda(), c.v_ctx.cuda(), c.cu_enc, c.kv_page_indptr,
+                          c.kv_page_indices, k_pool, v_pool)
+        plan = ctx.plan_paged(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len,
+                              num_pages)
+        outs.append(ctx.run_paged(plan, c.q.cuda(), k_pool, v_pool))
+    torch.cuda.synchronize()
+    ctx.check_device_status()
+    for c, o in zip(cases, outs):
+        assert_close(o, oracle_paged(c), what="double buffer")
+
+
+def test_stale_plan_is_rejected():
+    c = _case(210)
+    ctx = Context(8, 2, 64, 16)
+    kp, vp = gpu_pools(c, ctx)
+    p0 = ctx.plan_paged(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages, slot=0)
+    ctx.plan_paged(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages, slot=0)
+    with pytest.raises(ValueError, match="re-planned"):
+        ctx.run_paged(p0, c.q.cuda(), kp, vp)
+
+
+def test_plan_kind_must_match_run():
+    c = _case(211)
+    ctx = Context(8, 2, 64, 16)
+    kp, vp = gpu_pools(c, ctx)
+    rp = ctx.plan_ragged([0, 4], None, 0)
+    with pytest.raises(ValueError, match="kind"):
+        ctx.run_paged(rp, c.q.cuda(), kp, vp)
+
+
+def test_bad_tensors_are_rejected_before_launch():
+    c = _case(212)
+    ctx = Context(8, 2, 64, 16)
+    kp, vp = gpu_pools(c, ctx)
+    plan = ctx.plan_paged(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages)
+    with pytest.raises(ValueError):
+        ctx.run_paged(plan, c.q.cuda().float(), kp, vp)
+    with pytest.raises(ValueError):
+        ctx.run_paged(plan, c.q, kp, vp)          # host tensor
+    with pytest.raises(ValueError, match="UNSUPPORTED"):
+        Context(8, 3, 64, 16)
+
+
+def test_status_word_is_clear_after_normal_runs():
+    c = _case(213, qmax=20)
+    ctx = Context(8, 2, 64, 16)
+    kp, vp = gpu_pools(c, ctx)
+    plan = ctx.plan_paged(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages)
+    for _ in range(3):
+        ctx.run_paged(plan, c.q.cuda(), kp, vp)
+    ctx.check_device_status()
+    assert int(ctx.workspace[:4].view(torch.int32).item()) == 0

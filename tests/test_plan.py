@@ -1,0 +1,231 @@
+"""Host-side tests of the C-ABI library: symbol exports and the plan builder (no GPU).
+
+The plan must cover every visible (query token, query head, key) triple exactly once, keep
+its merge map consistent with its splits, reject malformed inputs, and be deterministic.
+"""
+import re
+import os
+
+import numpy as np
+import pytest
+
+from ragged_attention_encoder_b200 import _lib, build, inputs, plan_paged_host, plan_ragged_host
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="session", autouse=True)
+def built_library():
+    build.build()
+    return _lib.load()
+
+
+def test_library_exports_every_declared_symbol(built_library):
+    with open(os.path.join(ROOT, "include", "rae.h")) as f:
+        header = f.read()
+    declared = set(re.findall(r"^\s*(?:[\w\s\*]+?)\b(rae_\w+)\s*\(", header, flags=re.M))
+    assert len(declared) >= 15
+    assert declared == set(_lib.SIGNATURES), declared ^ set(_lib.SIGNATURES)
+    for name in declared:
+        assert hasattr(built_library, name), name
+
+
+def _tiles_rows(tiles, g):
+    """Expand tiles into (token, head, kv0, kv1, tile index)."""
+    out = []
+    for i, t in enumerate(tiles):
+        req, kvh, q0, qn, kv0, kv1, part, split = (int(x) for x in t)
+        for r in range(qn * g):
+            out.append((q0 + r // g, kvh * g + r % g, kv0, kv1, i))
+    return out
+
+
+def _check_cta_ptr(p):
+    cp = p["cta_ptr"]
+    raw = p["raw"]
+    assert cp[0] == 0 and cp[-1] == raw.num_tiles
+    assert np.all(np.diff(cp) >= 0)
+    if raw.num_tiles:
+        assert np.all(np.diff(cp) >= 1), "a launched CTA has no tile"
+
+
+def _check_merge(p, g, hq):
+    """Every split unit has one merge row per row, its splits tile the unit's partial rows."""
+    tiles = p["tiles"]
+    merge = p["merge"]
+    units = {}
+    for t in tiles:
+        req, kvh, q0, qn, kv0, kv1, part, split = (int(x) for x in t)
+        units.setdefault((req, kvh, q0), []).append((split, kv0, kv1, part, qn))
+    n_rows = 0
+    seen_parts = set()
+    for key, pieces in units.items():
+        pieces.sort()
+        assert [s for s, *_ in pieces] == list(range(len(pieces)))
+        for a, b in zip(pieces[:-1], pieces[1:]):
+            assert a[2] == b[1], "splits of a unit must be contiguous in keys"
+        qn = pieces[0][4]
+        if len(pieces) == 1:
+            assert pieces[0][3] == -1
+            continue
+        rows = qn * g
+        n_rows += rows
+        for s, kv0, kv1, part, _ in pieces:
+            assert part >= 0
+            for r in range(rows):
+                assert part + r not in seen_parts
+                seen_parts.add(part + r)
+        base = pieces[0][3]
+        req, kvh, q0 = key
+        for r in range(rows):
+            row = [m for m in merge if m[2] == base + r]
+            assert len(row) == 1
+            out_row, nsplit, part0, stride = (int(x) for x in row[0])
+            assert out_row == (q0 + r // g) * hq + kvh * g + r % g
+            assert nsplit == len(pieces) and stride == rows
+            for s, kv0, kv1, part, _ in pieces:
+                assert part == part0 - r + s * stride
+    assert n_rows == len(merge)
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("hq,hkv,d,P", [(4, 2, 64, 16), (8, 1, 128, 32), (6, 6, 64, 64),
+                                        (32, 8, 128, 16), (64, 8, 128, 64)])
+def test_paged_plan_covers_each_pair_once(seed, hq, hkv, d, P):
+    rng = np.random.default_rng(seed * 100 + hq)
+    B = int(rng.integers(1, 7))
+    q_len = rng.integers(0, 40 if seed % 2 else 3, B)
+    kv_len = rng.integers(0, 700, B)
+    pages_per = (kv_len + P - 1) // P + rng.integers(0, 2, B)
+    indptr = np.concatenate([[0], np.cumsum(pages_per)]).astype(np.int32)
+    num_pages = int(indptr[-1]) + 5
+    indices = rng.permutation(num_pages)[: indptr[-1]].astype(np.int32)
+    qo = np.concatenate([[0], np.cumsum(q_len)]).astype(np.int32)
+    # a small grid forces splits even on these small inputs
+    p = plan_paged_host(qo, indptr, indices, kv_len, num_pages, num_qo_heads=hq, num_kv_heads=hkv,
+                        head_dim=d, page_size=P, num_sms=int(rng.integers(1, 9)))
+    g = hq // hkv
+    _check_cta_ptr(p)
+    cover = {}
+    for tok, head, kv0, kv1, i in _tiles_rows(p["tiles"], g):
+        cover.setdefault((tok, head), []).append((kv0, kv1))
+    for b in range(B):
+        for tok in range(qo[b], qo[b + 1]):
+            for head in range(hq):
+                ranges = sorted(cover.pop((tok, head)))
+                keys = np.zeros(int(kv_len[b]), dtype=int)
+                for kv0, kv1 in ranges:
+                    assert 0 <= kv0 <= kv1 <= kv_len[b]
+                    keys[kv0:kv1] += 1
+                assert np.all(keys == 1)
+    assert not cover, "tiles cover rows that do not exist"
+    _check_merge(p, g, hq)
+
+
+@pytest.mark.parametrize("seed", range(4))
+@pytest.mark.parametrize("bs", [0, 1, 5, 128, 256])
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 2), (3, 1)])
+def test_ragged_plan_covers_each_visible_pair_once(seed, bs, hq, hkv):
+    rng = np.random.default_rng(seed + 7 * bs + hq)
+    S = int(rng.integers(1, 5))
+    lq = rng.integers(0, 300, S)
+    cross = seed % 2 == 1 and bs == 0
+    lk = rng.integers(0, 300, S) if cross else lq
+    cu_q = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
+    p = plan_ragged_host(cu_q, cu_k if cross else None, bs, num_qo_heads=hq, num_kv_heads=hkv,
+                         head_dim=128, num_sms=int(rng.integers(1, 5)))
+    g = hq // hkv
+    _check_cta_ptr(p)
+    cover = {}
+    for tok, head, kv0, kv1, i in _tiles_rows(p["tiles"], g):
+        cover.setdefault((tok, head), []).append((kv0, kv1))
+    for s in range(S):
+        for tok in range(cu_q[s], cu_q[s + 1]):
+            i_local = tok - cu_q[s]
+            # visible keys by the definition, enumerated one by one
+            vis = [j for j in range(int(lk[s])) if bs == 0 or (j // bs) <= (i_local // bs)]
+            for head in range(hq):
+                keys = np.zeros(int(lk[s]), dtype=int)
+                for kv0, kv1 in cover.pop((tok, head)):
+                    keys[kv0:kv1] += 1
+                assert np.all(keys[vis] == 1), "a visible key is not covered exactly once"
+                assert np.all(keys <= 1)
+    assert not cover
+    _check_merge(p, g, hq)
+
+
+def test_plan_is_deterministic():
+    c = inputs.workload(3)
+    kw = dict(num_qo_heads=32, num_kv_heads=8, head_dim=128, page_size=16)
+    a = plan_paged_host(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages, **kw)
+    b = plan_paged_host(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages, **kw)
+    for k in ("header", "cta_ptr", "tiles", "merge"):
+        assert np.array_equal(a[k], b[k])
+
+
+def test_plan_balances_the_grid():
+    c = inputs.workload(2)
+    p = plan_paged_host(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages,
+                        num_qo_heads=20, num_kv_heads=20, head_dim=64, page_size=16)
+    t, cp = p["tiles"], p["cta_ptr"]
+    load = np.array([int(((t[cp[i]:cp[i + 1], 5] - t[cp[i]:cp[i + 1], 4] + 15) // 16).sum() +
+                         2 * (cp[i + 1] - cp[i])) for i in range(p["raw"].num_ctas)])
+    assert p["raw"].num_ctas == 296
+    assert load.max() <= 1.02 * load[:-1].mean() + 2
+
+
+def test_decode_workloads_choose_the_simt_kernel():
+    kinds = {}
+    for i in (1, 2, 3, 5):
+        c = inputs.workload(i)
+        p = plan_paged_host(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len,
+                            c.num_pages, num_qo_heads=c.num_qo_heads, num_kv_heads=c.num_kv_heads,
+                            head_dim=c.head_dim, page_size=c.page_size)
+        kinds[i] = p["raw"].kind
+    assert kinds[1] == 1 and kinds[2] == 1 and kinds[3] == 2 and kinds[5] == 2
+
+
+@pytest.mark.parametrize("mutate,match", [
+    (lambda a: a.update(qo=np.array([0, 2, 1], np.int32)), "decreases"),
+    (lambda a: a.update(qo=np.array([1, 2, 3], np.int32)), r"\[0\] must be 0"),
+    (lambda a: a.update(idx=np.array([0, 1, 99], np.int32)), "outside"),
+    (lambda a: a.update(idx=np.array([0, -1, 2], np.int32)), "outside"),
+    (lambda a: a.update(kvl=np.array([16, 40], np.int32)), "fewer pages"),
+    (lambda a: a.update(kvl=np.array([-1, 3], np.int32)), "kv_len < 0"),
+])
+def test_invalid_paged_inputs_are_rejected(mutate, match):
+    a = dict(qo=np.array([0, 1, 2], np.int32), ip=np.array([0, 1, 3], np.int32),
+             idx=np.array([0, 1, 2], np.int32), kvl=np.array([16, 20], np.int32))
+    mutate(a)
+    with pytest.raises(ValueError, match=match):
+        plan_paged_host(a["qo"], a["ip"], a["idx"], a["kvl"], 4, num_qo_heads=4, num_kv_heads=2,
+                        head_dim=64, page_size=16)
+
+
+def test_unsupported_and_capacity_errors():
+    with pytest.raises(ValueError, match="UNSUPPORTED|unsupported"):
+        plan_paged_host([0, 1], [0, 1], [0], [3], 1, num_qo_heads=4, num_kv_heads=2, head_dim=96,
+                        page_size=16)
+    with pytest.raises(ValueError, match="CAPACITY"):
+        plan_paged_host([0, 1, 2], [0, 1, 2], [0, 1], [3, 3], 2, num_qo_heads=4, num_kv_heads=2,
+                        head_dim=64, page_size=16, max_batch=1)
+    with pytest.raises(ValueError, match="CAPACITY"):
+        plan_ragged_host([0, 300], None, 0, num_qo_heads=4, num_kv_heads=4, head_dim=64,
+                         max_q_tokens=100)
+
+
+def test_empty_inputs_plan_nothing():
+    p = plan_paged_host([0], [0], [], [], 1, num_qo_heads=4, num_kv_heads=2, head_dim=64,
+                        page_size=16)
+    assert p["raw"].num_tiles == 0 and p["raw"].num_ctas == 0
+    p = plan_paged_host([0, 0, 0], [0, 1, 2], [0, 1], [5, 9], 2, num_qo_heads=4, num_kv_heads=2,
+                        head_dim=64, page_size=16)
+    assert p["raw"].num_tiles == 0
+    p = plan_ragged_host([0, 0], None, 4, num_qo_heads=2, num_kv_heads=2, head_dim=64)
+    assert p["raw"].num_tiles == 0
+    # a request with queries but no context keys gets one empty tile (it writes zeros)
+    p = plan_paged_host([0, 2], [0, 0], [], [0], 1, num_qo_heads=4, num_kv_heads=2, head_dim=64,
+                        page_size=16)
+    t = p["tiles"]
+    assert t.shape[0] == 2 and np.all(t[:, 4] == 0) and np.all(t[:, 5] == 0)
