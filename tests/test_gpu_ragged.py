@@ -66,10 +66,12 @@ def test_two_span_cross_multitoken_shapes():
     assert_close(out, oracle_ragged(case), what="cross multitoken")
 
 
-def test_forced_splits_ragged():
-    case = inputs.ragged_case(130, span_lens=[700, 1500, 90], num_qo_heads=4, num_kv_heads=4,
-                              head_dim=128, block_size=256)
-    out, plan, *_ = run_ragged(case, num_sms=2)
+@pytest.mark.parametrize("bs,sms", [(256, 3), (0, 5)])
+def test_forced_splits_ragged(bs, sms):
+    """A small grid over few long units cuts some units' keys: split tiles plus the merge."""
+    case = inputs.ragged_case(130, span_lens=[1500, 700], num_qo_heads=1, num_kv_heads=1,
+                              head_dim=128, block_size=bs)
+    out, plan, *_ = run_ragged(case, num_sms=sms)
     assert plan.num_merge_rows > 0
     assert_close(out, oracle_ragged(case), what="ragged split")
 
