@@ -137,6 +137,28 @@ int rae_write_context(rae_ctx* ctx, const void* k_src, const void* v_src, const 
                       void* stream);
 
 /*
+ * Context write for callers that cannot allocate device memory.  The M* pages have no
+ * counterpart of this call.  It does what rae_write_context does (same arguments, layouts and
+ * validation; Hkv, head_dim and page_size given directly), but needs neither a context nor a
+ * workspace: its page-copy list goes to a 1 MiB array inside the library's own device memory,
+ * which every GPU that loads the library holds until the process exits.  It is meant for code
+ * whose device memory is owned by another allocator, or that must not call cudaMalloc (for
+ * example inside a latency-critical serving loop).  It calls no allocation routine.
+ *   - At most 65536 page copies (pages written) per call; more returns RAE_ERR_CAPACITY
+ *     before any device work.
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current); make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's list: calls that overlap on
+ *     the GPU (different streams, not ordered) race on it and must be serialised by the caller.
+ *   - The host arrays may be reused as soon as the call returns.
+ */
+int rae_write_context_noalloc(const void* k_src, const void* v_src, const int32_t* cu_enc,
+                              const int32_t* page_indptr, const int32_t* page_indices,
+                              int32_t batch, void* k_pool, void* v_pool, int32_t num_pages,
+                              int32_t num_kv_heads, int32_t head_dim, int32_t page_size,
+                              void* stream);
+
+/*
  * Plan of paged cross-attention (FlashInferCrossManager.plan; QueryPacking.qo_indptr).
  * Host int32 arrays: qo_indptr [B+1] (cumulative query lengths, qo_indptr[0] == 0),
  * kv_page_indptr [B+1], kv_page_indices [kv_page_indptr[B]], kv_len [B] (context tokens of

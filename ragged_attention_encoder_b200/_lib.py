@@ -93,6 +93,8 @@ SIGNATURES = {
     "rae_plan_ragged_host": (ctypes.c_int, [ctypes.POINTER(RaeConfig), P32, P32, i32, i32, vp,
                                             sz, ctypes.POINTER(RaePlan), ctypes.c_char_p, sz]),
     "rae_plan_image_bytes_for": (sz, [ctypes.POINTER(RaeConfig)]),
+    "rae_write_context_noalloc": (ctypes.c_int, [vp, vp, P32, P32, P32, i32, vp, vp, i32, i32,
+                                                 i32, i32, vp]),
     "rae_enable_kernel_timing": (ctypes.c_int, [vp, i32]),
     "rae_read_kernel_timing": (ctypes.c_int, [vp, ctypes.POINTER(ctypes.c_float),
                                               ctypes.POINTER(ctypes.c_float), i32,

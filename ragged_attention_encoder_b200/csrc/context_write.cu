@@ -6,7 +6,11 @@
 // one contiguous block of ntok * Hkv * d elements, the destination is the page's Hkv runs of
 // ntok * d elements, so both sides move in whole 16-byte vectors with coalesced accesses.
 // HBM bound: algorithmic bytes = 2 (K and V) x 2 (read + write) x tokens x Hkv x d x 2 B.
+#include <mutex>
+#include <string>
+
 #include "kernels.h"
+#include "rae.h"
 
 namespace rae {
 namespace {
@@ -50,3 +54,88 @@ cudaError_t launch_context_write(const WriteItem* items, int64_t num_items, cons
 }
 
 }  // namespace rae
+
+// ---------------------------------------------------------------------------------------
+// Context write without a caller workspace (rae_write_context_noalloc).
+//
+// The ordinary call stages its page-copy list in the caller's workspace.  Some callers have
+// no way to provide one: a serving engine whose device memory is owned entirely by its own
+// pool allocator, or code that must not call cudaMalloc at all (because an allocation would
+// stall a latency-critical loop or fall outside the memory budget it was given).  For them
+// the list lives in this file-scope device array instead.  Every GPU that loads the library
+// holds the array (1 MiB) until the process exits.
+namespace rae {
+namespace {
+
+constexpr int64_t kNoAllocMaxPages = 65536;   // page copies per call (16 B each)
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) WriteItem g_noalloc_items[kNoAllocMaxPages];
+
+WriteItem g_noalloc_host[kNoAllocMaxPages];            // host-side build of the list
+WriteItem* g_noalloc_dev[kNoAllocMaxDevices] = {};     // device address of the array, per GPU
+std::mutex g_noalloc_mutex;
+
+}  // namespace
+}  // namespace rae
+
+extern "C" int rae_write_context_noalloc(const void* k_src, const void* v_src,
+                                         const int32_t* cu_enc, const int32_t* page_indptr,
+                                         const int32_t* page_indices, int32_t batch,
+                                         void* k_pool, void* v_pool, int32_t num_pages,
+                                         int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t page_size, void* stream) {
+  using namespace rae;
+  if (!k_pool || !v_pool) return RAE_ERR_INVALID_ARG;
+  const uintptr_t mis = reinterpret_cast<uintptr_t>(k_src) | reinterpret_cast<uintptr_t>(v_src) |
+                        reinterpret_cast<uintptr_t>(k_pool) | reinterpret_cast<uintptr_t>(v_pool);
+  if (mis & 15) return RAE_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RAE_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return RAE_ERR_UNSUPPORTED;
+
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_dev[dev]) {
+    // Once per device, with that device current: the host-side name of the array is only a
+    // stand-in, the kernel needs the address the runtime gives for this device.
+    void* addr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_items);
+    if (e != cudaSuccess || !addr) return RAE_ERR_CUDA;
+    g_noalloc_dev[dev] = static_cast<WriteItem*>(addr);
+  }
+
+  rae_config cfg{};
+  cfg.num_qo_heads = num_kv_heads;
+  cfg.num_kv_heads = num_kv_heads;
+  cfg.head_dim = head_dim;
+  cfg.page_size = page_size;
+  cfg.max_batch = batch > 0 ? batch : 1;
+  cfg.max_q_tokens = 1;
+  cfg.max_kv_pages = int32_t(kNoAllocMaxPages);
+  cfg.max_tiles = 1;
+  cfg.max_partial_rows = 0;
+  cfg.num_sms = 1;
+  int64_t n = 0;
+  std::string msg;
+  // Sizes beyond kNoAllocMaxPages page copies come back as RAE_ERR_CAPACITY, before any
+  // device work.
+  int rc = build_write_items(cfg, cu_enc, page_indptr, page_indices, batch, num_pages,
+                             g_noalloc_host, kNoAllocMaxPages, &n, &msg);
+  if (rc) return rc;
+  if (n == 0) return RAE_OK;
+  if (!k_src || !v_src) return RAE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // From pageable host memory: the call returns once the list has been staged, so the host
+  // array may be rebuilt by the next call.
+  cudaError_t e = cudaMemcpyAsync(g_noalloc_dev[dev], g_noalloc_host,
+                                  size_t(n) * sizeof(WriteItem), cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return RAE_ERR_CUDA;
+  Geometry geo;
+  geo.hq = num_kv_heads;
+  geo.hkv = num_kv_heads;
+  geo.g = 1;
+  geo.d = head_dim;
+  geo.page_size = page_size;
+  e = launch_context_write(g_noalloc_dev[dev], n, k_src, v_src, k_pool, v_pool, geo, st);
+  return e == cudaSuccess ? RAE_OK : RAE_ERR_CUDA;
+}
