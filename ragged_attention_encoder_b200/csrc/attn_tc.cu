@@ -1,54 +1,59 @@
-// Tensor-core attention over 128-row query tiles for sm_100a (tcgen05 + TMEM + TMA).
+// Tensor-core attention for sm_100a (tcgen05 + TMEM + TMA), two query tiles per CTA.
 //
 // Serves the paged cross-attention of multi-token query packs (M* page
 // "mstar.engine.resources.attn.cross", FlashInferCrossManager.run: non-causal over the
 // context) and the cacheless ragged attentions (page "mstar.engine.resources.attn.ragged.base":
 // block-causal self-attention within a span, and two-span cross-attention).
 //
-// A tile is up to 128 query rows of one (request, KV head): rows are (token, head in group)
-// pairs, so the g = Hq/Hkv query heads that share a KV head share every K/V byte loaded.
-// Per 128-key block j of the tile's key range:
-//     S   = Q K^T                     tcgen05.mma, M=128 N=128, fp32 accumulators in TMEM
-//     P   = exp2(S*scale*log2e - m)   one thread per row (TMEM lane), fp32, online max
-//     O  += P V                       tcgen05.mma, M=128 N=d, P staged as bf16 in smem
-// and the epilogue writes O / l as bf16 (or an fp32 partial and its log2-sum-exp when the
-// plan split the unit's keys).  The row sum l is accumulated from the bf16-rounded P that
-// the tensor core multiplies, so a constant V comes back exactly.
+// A work tile holds up to two 128-row query tiles Q0, Q1 of one (request, KV head) with one
+// key range, so every K/V block loaded serves 256 query rows.  Rows are (token, head in
+// group) pairs: the g = Hq/Hkv heads of a KV head share each K/V byte.  Per 128-key block j:
+//     S_t = Q_t K_j^T                    tcgen05.mma M=128 N=128, fp32 accumulators in TMEM
+//     P_t = exp2(S_t*scale*log2e - m_t)  one thread per row, fp32, written back into TMEM as
+//                                        bf16 over the first half of S_t's columns
+//     O_t += P_t V_j                     tcgen05.mma with A = P_t read from TMEM, N = d
+// The MMA warp interleaves the two tiles (S0 S1 | PV0 S0' | PV1 S1' | ...) so that the tensor
+// core works on one tile while the other tile's softmax runs.  O is rescaled only when a row's
+// maximum grows by more than 2^8 (the exponent base stays stale otherwise, which is exact
+// after the final division).  The row sum l is accumulated from the bf16-rounded P that the
+// tensor core multiplies, so a constant V comes back exactly.
 //
-// Warp roles (192 threads): warps 0-3 softmax + epilogue (warp w owns TMEM lanes 32w..32w+31),
-// warp 4 TMA producer, warp 5 MMA issuer (one thread) and TMEM owner.  K/V blocks stream
-// through a 2-stage ring; S of block j+1 is computed while the softmax of block j runs.
-// Masking is by select (never by adding): keys past the row's limit get -inf, and V rows past
-// the valid keys of the last block are zeroed in shared memory before P.V, so junk (even NaN)
-// in page tails cannot reach the output.
+// Warp roles (320 threads): warps 0-3 softmax + epilogue of Q0 (TMEM lanes 32w..32w+31),
+// warps 4-7 the same for Q1, warp 8 TMA producer, warp 9 MMA issuer and TMEM owner.
+// Masking is by select: keys past a row's limit get -inf, and V rows past the valid keys of
+// the last block are zeroed in shared memory before P.V, so junk (even NaN) in page tails
+// cannot reach the output.  Every wait is bounded.
 #include "kernels.h"
 #include "ptx.cuh"
 
 namespace rae {
 namespace {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr int kStages = 2;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kSCol = 0;
-constexpr uint32_t kOCol = 128;
+constexpr uint32_t kTmemCols = 512;
 constexpr int kChunkBytes = 128 * 128;   // 128 rows x 64 bf16 (one 128-byte swizzle span)
 
 template <int D>
 struct TcLayout {
   static constexpr int CH = D / 64;
-  static constexpr int TILE = CH * kChunkBytes;   // Q, K or V tile bytes
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = TILE;
+  static constexpr int TILE = CH * kChunkBytes;   // bytes of a 128-row Q, K or V tile
+  static constexpr int Q_OFF = 0;                  // Q0, Q1
+  static constexpr int K_OFF = 2 * TILE;
   static constexpr int V_OFF = K_OFF + kStages * TILE;
-  static constexpr int P_OFF = V_OFF + kStages * TILE;
-  static constexpr int BAR_OFF = P_OFF + 2 * kChunkBytes;
-  static constexpr int SMEM = BAR_OFF + 256 + 1024;   // barriers + alignment slack
+  static constexpr int BAR_OFF = V_OFF + kStages * TILE;
+  static constexpr int SMEM = BAR_OFF + 512 + 1024;   // barriers + alignment slack
+  // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 after it.
+  static __device__ __forceinline__ constexpr uint32_t s_col(int qt) { return uint32_t(qt) * 128u; }
+  static __device__ __forceinline__ constexpr uint32_t o_col(int qt) { return 256u + uint32_t(qt) * D; }
 };
 
 struct TcBars {
-  uint64_t q_full, q_empty, s_full, s_free, p_full, pv_done, o_free, fin;
-  uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+  uint64_t q_full, q_empty, fin;
+  uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
+  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   uint32_t tmem_base;
   int abort;
 };
@@ -70,6 +75,54 @@ __device__ __forceinline__ int tile_blocks(const Tile& t) {
   return (t.kv1 - t.kv0 + kTcBlockKeys - 1) / kTcBlockKeys;
 }
 
+// D[tmem] (+)= A[tmem] * B[smem], kind::f16 (A = P in TMEM, bf16 pairs per 32-bit column).
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// S = Q K^T for one 128-row tile: D/16 MMAs of K=16 over the 128-byte-swizzled K-major tiles.
+template <int D>
+__device__ __forceinline__ void mma_s(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr,
+                                      uint32_t idesc) {
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const uint32_t off = (ks >> 2) * kChunkBytes + (ks & 3) * 32;
+    umma_ss(d_tmem, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
+            idesc, ks > 0 ? 1u : 0u);
+  }
+}
+
+// O (+)= P V for one tile: P (128 x 128 keys, bf16 pairs) from TMEM, V MN-major from smem.
+template <int D>
+__device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_addr,
+                                       uint32_t idesc, bool first) {
+#pragma unroll
+  for (int ks = 0; ks < kTcBlockKeys / 16; ++ks)
+    umma_ts(o_tmem, p_tmem + ks * 8, smem_desc_sw128(v_addr + ks * 16 * 128, kChunkBytes, 1024),
+            idesc, (ks > 0 || !first) ? 1u : 0u);
+}
+
+// O row *= f, 16 columns at a time (rare: only when a row's maximum grew by more than 2^8).
+// Kept out of line so that its registers do not add to the softmax loop's.
+template <int D>
+__device__ __noinline__ void rescale_o(uint32_t o_addr, float f) {
+#pragma unroll 1
+  for (int c = 0; c < D / 16; ++c) {
+    uint32_t ov[16];
+    tmem_ld16(o_addr + c * 16, ov);
+    tmem_wait_ld(ov);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+    tmem_st16(o_addr + c * 16, ov);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
   using L = TcLayout<D>;
@@ -85,25 +138,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
   if (threadIdx.x == 0) {
     mbar_init(&bar.q_full, 1);
     mbar_init(&bar.q_empty, 1);
-    mbar_init(&bar.s_full, 1);
-    mbar_init(&bar.s_free, 4);
-    mbar_init(&bar.p_full, 4);
-    mbar_init(&bar.pv_done, 1);
-    mbar_init(&bar.o_free, 4);
     mbar_init(&bar.fin, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bar.s_full[t], 1);
+      mbar_init(&bar.p_full[t], 4);
+      mbar_init(&bar.pv_done[t], 1);
+      mbar_init(&bar.o_free[t], 4);
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar.k_full[s], 1);
+      mbar_init(&bar.k_empty[s], 1);
       mbar_init(&bar.v_full[s], 1);
-      mbar_init(&bar.kv_empty[s], 1);
+      mbar_init(&bar.v_empty[s], 1);
     }
     bar.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bar.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&p.maps.q);
     prefetch_tmap(&p.maps.k);
     prefetch_tmap(&p.maps.v);
@@ -117,63 +172,65 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
   const int t_begin = plan.cta_ptr[blockIdx.x];
   const int t_end = plan.cta_ptr[blockIdx.x + 1];
   const int g = geo.g;
-  const int tpt = kTcRows / g;   // query tokens per tile
+  const int tpt = kTcRows / g;   // query tokens per 128-row tile
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ================================================================ TMA producer
     if (lane == 0) {
       const uint64_t pol_q = policy_evict_first();
       const uint64_t pol_kv = policy_evict_last();
-      const uint32_t q_bytes = uint32_t(L::CH) * 64u * 2u * uint32_t(g * tpt);
+      const uint32_t q_tile_bytes = uint32_t(L::CH) * 64u * 2u * uint32_t(g * tpt);
       uint32_t q_use = 0, kv_use = 0;
       for (int t = t_begin; t < t_end && !bar.abort; ++t) {
         const Tile tile = plan.tiles[t];
         const int n = tile_blocks(tile);
         if (n == 0) continue;
+        const bool has1 = tile.qn > tpt;
         if (q_use > 0 && !wait_bounded(&bar.q_empty, (q_use - 1) & 1, wc, 201)) break;
-        mbar_arrive_expect_tx(&bar.q_full, q_bytes);
-        for (int c = 0; c < L::CH; ++c)
-          tma_load_3d(smem + L::Q_OFF + c * kChunkBytes, &p.maps.q, &bar.q_full, c * 64,
-                      tile.kv_head * g, tile.q0, pol_q);
+        mbar_arrive_expect_tx(&bar.q_full, q_tile_bytes * (has1 ? 2u : 1u));
+        for (int qt = 0; qt < (has1 ? 2 : 1); ++qt)
+          for (int c = 0; c < L::CH; ++c)
+            tma_load_3d(smem + L::Q_OFF + qt * L::TILE + c * kChunkBytes, &p.maps.q, &bar.q_full,
+                        c * 64, tile.kv_head * g, tile.q0 + qt * tpt, pol_q);
         ++q_use;
         const int32_t* pages = p.paged ? plan.d + plan.c[tile.req] : nullptr;
         const int32_t kv_base = p.paged ? 0 : plan.b[tile.req];
         bool ok = true;
         for (int j = 0; j < n; ++j, ++kv_use) {
           const int s = kv_use % kStages;
-          if (kv_use >= uint32_t(kStages) &&
-              !wait_bounded(&bar.kv_empty[s], ((kv_use / kStages) - 1) & 1, wc, 202)) {
-            ok = false;
-            break;
-          }
+          const uint32_t ph = ((kv_use / kStages) - 1) & 1;
           const int key0 = tile.kv0 + j * kTcBlockKeys;
           uint8_t* ks = smem + L::K_OFF + s * L::TILE;
           uint8_t* vs = smem + L::V_OFF + s * L::TILE;
+          if (kv_use >= uint32_t(kStages) && !wait_bounded(&bar.k_empty[s], ph, wc, 202)) { ok = false; break; }
           if (p.paged) {
             const int P = geo.page_size;
             const int nk = min(kTcBlockKeys, tile.kv1 - key0);
             const int npg = (nk + P - 1) / P;
             const uint32_t bytes = uint32_t(npg) * uint32_t(P) * 128u * L::CH;
             mbar_arrive_expect_tx(&bar.k_full[s], bytes);
+            for (int i = 0; i < npg; ++i) {
+              const int row = (pages[key0 / P + i] * geo.hkv + tile.kv_head) * P;
+              for (int c = 0; c < L::CH; ++c)
+                tma_load_2d(ks + c * kChunkBytes + i * P * 128, &p.maps.k, &bar.k_full[s], c * 64, row, pol_kv);
+            }
+            if (kv_use >= uint32_t(kStages) && !wait_bounded(&bar.v_empty[s], ph, wc, 203)) { ok = false; break; }
             mbar_arrive_expect_tx(&bar.v_full[s], bytes);
             for (int i = 0; i < npg; ++i) {
-              const int page = pages[key0 / P + i];
-              const int row = (page * geo.hkv + tile.kv_head) * P;
-              for (int c = 0; c < L::CH; ++c) {
-                tma_load_2d(ks + c * kChunkBytes + i * P * 128, &p.maps.k, &bar.k_full[s], c * 64, row, pol_kv);
+              const int row = (pages[key0 / P + i] * geo.hkv + tile.kv_head) * P;
+              for (int c = 0; c < L::CH; ++c)
                 tma_load_2d(vs + c * kChunkBytes + i * P * 128, &p.maps.v, &bar.v_full[s], c * 64, row, pol_kv);
-              }
             }
           } else {
-            const uint32_t bytes = uint32_t(L::TILE);
-            mbar_arrive_expect_tx(&bar.k_full[s], bytes);
-            mbar_arrive_expect_tx(&bar.v_full[s], bytes);
-            for (int c = 0; c < L::CH; ++c) {
+            mbar_arrive_expect_tx(&bar.k_full[s], uint32_t(L::TILE));
+            for (int c = 0; c < L::CH; ++c)
               tma_load_3d(ks + c * kChunkBytes, &p.maps.k, &bar.k_full[s], c * 64, tile.kv_head,
                           kv_base + key0, pol_kv);
+            if (kv_use >= uint32_t(kStages) && !wait_bounded(&bar.v_empty[s], ph, wc, 203)) { ok = false; break; }
+            mbar_arrive_expect_tx(&bar.v_full[s], uint32_t(L::TILE));
+            for (int c = 0; c < L::CH; ++c)
               tma_load_3d(vs + c * kChunkBytes, &p.maps.v, &bar.v_full[s], c * 64, tile.kv_head,
                           kv_base + key0, pol_kv);
-            }
           }
         }
         if (!ok) break;
@@ -194,70 +251,75 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-      const uint32_t q_addr = sbase + L::Q_OFF;
-      const uint32_t p_addr = sbase + L::P_OFF;
-      uint32_t q_use = 0, kv_use = 0, blk = 0, o_waits = 0, tiles_done = 0;
-      // The P.V of block b is issued after the QK^T of block b+1, so that the tensor core
-      // computes the next scores while the softmax of block b runs.
-      bool have_prev = false, prev_first = false, prev_wait_o = false;
-      uint32_t prev_blk = 0, prev_use = 0;
-      auto issue_pv = [&]() -> bool {
-        if (!wait_bounded(&bar.p_full, prev_blk & 1, wc, 211)) return false;
-        const int s = prev_use % kStages;
-        if (!wait_bounded(&bar.v_full[s], (prev_use / kStages) & 1, wc, 212)) return false;
-        if (prev_wait_o) {
-          if (!wait_bounded(&bar.o_free, o_waits & 1, wc, 213)) return false;
-          ++o_waits;
-        }
-        tc_fence_after();
-        const uint32_t v_addr = sbase + L::V_OFF + s * L::TILE;
-#pragma unroll
-        for (int ks = 0; ks < kTcBlockKeys / 16; ++ks) {
-          const uint64_t a = smem_desc_sw128(p_addr + (ks >> 2) * kChunkBytes + (ks & 3) * 32, 16, 1024);
-          const uint64_t b = smem_desc_sw128(v_addr + ks * 16 * 128, kChunkBytes, 1024);
-          umma_ss(tmem + kOCol, a, b, idesc_pv, (ks > 0 || !prev_first) ? 1u : 0u);
-        }
-        umma_commit(&bar.kv_empty[s]);
-        umma_commit(&bar.pv_done);
-        return true;
-      };
+      uint32_t q_use = 0, kv_use = 0;
+      uint32_t pv_cnt0 = 0, pv_cnt1 = 0, o_tiles0 = 0, o_tiles1 = 0;
       bool ok = true;
       for (int t = t_begin; t < t_end && ok; ++t) {
         const Tile tile = plan.tiles[t];
         const int n = tile_blocks(tile);
         if (n == 0) continue;
+        const bool has1 = tile.qn > tpt;
         if (!wait_bounded(&bar.q_full, q_use & 1, wc, 214)) { ok = false; break; }
         ++q_use;
-        for (int j = 0; j < n; ++j, ++kv_use, ++blk) {
+        // Prologue: S of block 0 for both tiles.
+        {
           const int s = kv_use % kStages;
           if (!wait_bounded(&bar.k_full[s], (kv_use / kStages) & 1, wc, 215)) { ok = false; break; }
-          if (blk > 0 && !wait_bounded(&bar.s_free, (blk - 1) & 1, wc, 216)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t k_addr = sbase + L::K_OFF + s * L::TILE;
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * kChunkBytes + (ks & 3) * 32;
-            const uint64_t a = smem_desc_sw128(q_addr + off, 16, 1024);
-            const uint64_t b = smem_desc_sw128(k_addr + off, 16, 1024);
-            umma_ss(tmem + kSCol, a, b, idesc_qk, ks > 0 ? 1u : 0u);
+          for (int qt = 0; qt < 2; ++qt) {
+            if (qt == 1 && !has1) break;
+            mma_s<D>(tmem + L::s_col(qt), sbase + L::Q_OFF + qt * L::TILE,
+                     sbase + L::K_OFF + s * L::TILE, idesc_qk);
+            umma_commit(&bar.s_full[qt]);
           }
-          umma_commit(&bar.s_full);
-          if (j == n - 1) umma_commit(&bar.q_empty);
-          if (have_prev && !issue_pv()) { ok = false; break; }
-          have_prev = true;
-          prev_blk = blk;
-          prev_use = kv_use;
-          prev_first = (j == 0);
-          prev_wait_o = (j == 0 && tiles_done > 0);
+          umma_commit(&bar.k_empty[s]);
+          if (n == 1) umma_commit(&bar.q_empty);
         }
-        ++tiles_done;
+        for (int j = 0; j < n && ok; ++j) {
+          const uint32_t use = kv_use + j;
+          const int s = use % kStages;
+          const int s1 = (use + 1) % kStages;
+          const bool more = j + 1 < n;
+          if (!wait_bounded(&bar.v_full[s], (use / kStages) & 1, wc, 212)) { ok = false; break; }
+          if (more && !wait_bounded(&bar.k_full[s1], ((use + 1) / kStages) & 1, wc, 216)) { ok = false; break; }
+#pragma unroll
+          for (int qt = 0; qt < 2; ++qt) {
+            if (qt == 1 && !has1) break;
+            const uint32_t o_tiles = qt ? o_tiles1 : o_tiles0;
+            const uint32_t pv_cnt = qt ? pv_cnt1 : pv_cnt0;
+            // The first P.V of a tile overwrites O: the previous tile's epilogue must have
+            // read it out.
+            if (j == 0 && o_tiles > 0 &&
+                !wait_bounded(&bar.o_free[qt], (o_tiles - 1) & 1, wc, 213)) { ok = false; break; }
+            if (!wait_bounded(&bar.p_full[qt], pv_cnt & 1, wc, 211)) { ok = false; break; }
+            tc_fence_after();
+            mma_pv<D>(tmem + L::o_col(qt), tmem + L::s_col(qt), sbase + L::V_OFF + s * L::TILE,
+                      idesc_pv, j == 0);
+            umma_commit(&bar.pv_done[qt]);
+            if (qt) ++pv_cnt1; else ++pv_cnt0;
+            if (more) {   // after P_qt(j) was consumed (the tensor pipe runs in issue order)
+              mma_s<D>(tmem + L::s_col(qt), sbase + L::Q_OFF + qt * L::TILE,
+                       sbase + L::K_OFF + s1 * L::TILE, idesc_qk);
+              umma_commit(&bar.s_full[qt]);
+            }
+          }
+          if (!ok) break;
+          umma_commit(&bar.v_empty[s]);
+          if (more) {
+            umma_commit(&bar.k_empty[s1]);
+            if (j + 2 == n) umma_commit(&bar.q_empty);
+          }
+        }
+        kv_use += n;
+        ++o_tiles0;
+        if (has1) ++o_tiles1;
       }
-      if (ok && have_prev) issue_pv();
       // Every issued MMA completes before TMEM is released.
       umma_commit(&bar.fin);
       const uint64_t t0 = global_timer_ns();
@@ -266,17 +328,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
     }
   } else {
     // ================================================================ softmax + epilogue
-    const int r = warp * 32 + lane;               // tile row == TMEM lane
-    const uint32_t lane_addr = tmem + (uint32_t(warp * 32) << 16);
-    const int tok = r / g;
-    const int jh = r - tok * g;
-    uint32_t kv_use = 0, blk = 0;
+    const int qt = warp >> 2;                     // query tile of this warpgroup
+    const int wq = warp & 3;                      // TMEM lane quadrant
+    const int r = wq * 32 + lane;                 // row of the tile == TMEM lane
+    const uint32_t lane_addr = tmem + (uint32_t(wq * 32) << 16);
+    const uint32_t s_col = L::s_col(qt);
+    const uint32_t o_col = L::o_col(qt);
+    const int tok_in_tile = r / g;
+    const int jh = r - tok_in_tile * g;
+    uint32_t kv_use = 0, s_cnt = 0, pv_cnt = 0;
     for (int t = t_begin; t < t_end; ++t) {
       const Tile tile = plan.tiles[t];
       const int n = tile_blocks(tile);
+      const bool has1 = tile.qn > tpt;
+      if (qt == 1 && !has1) {
+        kv_use += n;
+        continue;
+      }
+      const int tok = qt * tpt + tok_in_tile;     // token index within the work tile
       const bool row_ok = tok < tile.qn && r < tpt * g;
       const int q_tok = tile.q0 + tok;
       const int head = tile.kv_head * g + jh;
+      const int urow = tok * g + jh;               // row within the unit (partials)
       // Keys visible to this row, as a limit on the logical key index.
       int lim = tile.kv1;
       if (!p.paged) {
@@ -291,107 +364,96 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       }
       float m = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < n; ++j, ++kv_use, ++blk) {
-        const int s = kv_use % kStages;
-        ok = __all_sync(0xffffffffu, wait_bounded(&bar.s_full, blk & 1, wc, 221));
+      for (int j = 0; j < n; ++j) {
+        const uint32_t use = kv_use + j;
+        ok = __all_sync(0xffffffffu, wait_bounded(&bar.s_full[qt], s_cnt & 1, wc, 221));
         if (!ok) break;
+        ++s_cnt;
         tc_fence_after();
-        uint32_t sv[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + kSCol + c * 32, sv[c]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_wait_ld(sv[c]);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar.s_free);
-
         const int key0 = tile.kv0 + j * kTcBlockKeys;
         const int nv = max(0, min(kTcBlockKeys, lim - key0));
-        float mx = -INFINITY;
+        // Row maximum of the raw scores with independent partial maxima (no serial chain);
+        // keys past the row's limit become -inf (only in blocks that have any).
+        const bool full = __all_sync(0xffffffffu, nv == kTcBlockKeys);
+        uint32_t sv[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + s_col + c * 32, sv[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_wait_ld(sv[c]);
+        if (!full) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (c * 32 + e >= nv) sv[c][e] = __float_as_uint(-INFINITY);
+        }
+        float pm[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pm[i] = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int col = c * 32 + e;
-            const float x = col < nv ? __uint_as_float(sv[c][e]) * p.scale_log2 : -INFINITY;
-            sv[c][e] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
-          }
+          for (int e = 0; e < 32; ++e) pm[e & 7] = fmaxf(pm[e & 7], __uint_as_float(sv[c][e]));
+        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * p.scale_log2;
         const float mn = fmaxf(m, mx);
-        // Rescale lazily: keep the old maximum unless the new one exceeds it by 2^8.
-        const bool need = (j == 0) ? true : (mn > m + 8.f);
-        const bool warp_need = __any_sync(0xffffffffu, need && j > 0);
-        float m_use = need ? mn : m;
-        const float corr = (need && m != -INFINITY && mn != -INFINITY) ? fast_exp2(m - mn)
-                                                                      : (need && j > 0 ? 0.f : 1.f);
-        const float base = (m_use == -INFINITY) ? 0.f : m_use;
-        float psum = 0.f;
-        uint32_t pk[64];
+        // Keep the old maximum unless the new one exceeds it by 2^8 (exact after division).
+        const bool need = (j == 0) || (mn > m + 8.f);
+        const bool rescale = j > 0 && need && m != -INFINITY;
+        const float corr = rescale ? fast_exp2(m - mn) : 1.f;
+        if (need) m = mn;
+        const float nbase = (m == -INFINITY) ? 0.f : -m;
+        // p = 2^(s * scale - m) rounded to bf16 and stored over the first 64 columns of S;
+        // the row sum adds exactly those bf16 values.
+        uint64_t ps[2] = {0, 0};
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float p0 = fast_exp2(__uint_as_float(sv[c][e]) - base);
-            const float p1 = fast_exp2(__uint_as_float(sv[c][e + 1]) - base);
-            const uint32_t w = pack_bf16x2(p0, p1);
-            pk[c * 16 + e / 2] = w;
-            psum += bf16lo_to_f32(w) + bf16hi_to_f32(w);
+          for (int e = 0; e < 16; ++e) {
+            pk[e] = pack_bf16x2(fast_exp2(fmaf(__uint_as_float(sv[c][2 * e]), p.scale_log2, nbase)),
+                                fast_exp2(fmaf(__uint_as_float(sv[c][2 * e + 1]), p.scale_log2, nbase)));
+            ps[e & 1] = f32x2_add(ps[e & 1], bf16x2_to_f32x2(pk[e]));
           }
-        if (blk > 0) {
-          ok = __all_sync(0xffffffffu, wait_bounded(&bar.pv_done, (blk - 1) & 1, wc, 222));
+          tmem_st16(lane_addr + s_col + c * 16, pk);
+        }
+        const float psum = f32x2_sum(ps[0]) + f32x2_sum(ps[1]);
+        l = l * corr + psum;
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O holds the sum through block j-1 once P.V of block j-1 has completed.
+          ok = __all_sync(0xffffffffu, wait_bounded(&bar.pv_done[qt], (pv_cnt + j - 1) & 1, wc, 222));
           if (!ok) break;
-        }
-        if (warp_need) {
           tc_fence_after();
-          const float cf = (need && j > 0) ? corr : 1.f;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(lane_addr + kOCol + c * 32, ov);
-            tmem_wait_ld(ov);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * cf);
-            tmem_st32(lane_addr + kOCol + c * 32, ov);
-          }
-          tmem_wait_st();
+          rescale_o<D>(lane_addr + o_col, corr);
         }
-        l = (j > 0 && need) ? l * corr + psum : (j == 0 ? psum : l + psum);
-        m = m_use;
-        // P row r -> bf16, 128-byte swizzled K-major layout (two 64-key chunks).
-        uint8_t* prow = smem + L::P_OFF + r * 128;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int chunk = u >> 3, w = u & 7;
-          uint4 v;
-          v.x = pk[u * 4 + 0];
-          v.y = pk[u * 4 + 1];
-          v.z = pk[u * 4 + 2];
-          v.w = pk[u * 4 + 3];
-          *reinterpret_cast<uint4*>(prow + chunk * kChunkBytes + ((w ^ (r & 7)) << 4)) = v;
-        }
-        // V rows past the block's valid keys hold stale or junk data: zero them.
+        tmem_wait_st();
+        // V rows past the block's valid keys hold stale or junk data: zero them (the first
+        // tile's warpgroup does it; P.V of either tile is issued after its p_full).
         const int vb = min(kTcBlockKeys, tile.kv1 - key0);
-        if (r >= vb) {
-          if (wait_bounded(&bar.v_full[s], (kv_use / kStages) & 1, wc, 223)) {
+        if (qt == 0 && r >= vb) {
+          const int s = use % kStages;
+          if (wait_bounded(&bar.v_full[s], (use / kStages) & 1, wc, 223)) {
             uint8_t* vrow = smem + L::V_OFF + s * L::TILE + r * 128;
 #pragma unroll
             for (int c = 0; c < L::CH; ++c)
 #pragma unroll
               for (int u = 0; u < 8; ++u)
                 *reinterpret_cast<uint4*>(vrow + c * kChunkBytes + u * 16) = make_uint4(0, 0, 0, 0);
+            fence_proxy_async_smem();
           }
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar.p_full);
+        if (lane == 0) mbar_arrive(&bar.p_full[qt]);
       }
       if (!ok) break;
+      kv_use += n;
       // ---------------------------------------------------------------- epilogue
       const bool split = tile.part >= 0;
       if (n > 0) {
-        ok = __all_sync(0xffffffffu, wait_bounded(&bar.pv_done, (blk - 1) & 1, wc, 224));
+        ok = __all_sync(0xffffffffu, wait_bounded(&bar.pv_done[qt], (pv_cnt + n - 1) & 1, wc, 224));
         if (!ok) break;
+        pv_cnt += n;
         tc_fence_after();
       }
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -399,7 +461,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
         if (n > 0) {
-          tmem_ld32(lane_addr + kOCol + c * 32, ov);
+          tmem_ld32(lane_addr + o_col + c * 32, ov);
           tmem_wait_ld(ov);
         } else {
 #pragma unroll
@@ -415,25 +477,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
         } else {
-          float4* dst = reinterpret_cast<float4*>(p.part_o + int64_t(tile.part + r) * D + c * 32);
+          float4* dst = reinterpret_cast<float4*>(p.part_o + int64_t(tile.part + urow) * D + c * 32);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
                                  __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
         }
       }
-      if (split && row_ok) p.part_lse[tile.part + r] = l > 0.f ? m + fast_log2(l) : -INFINITY;
+      if (split && row_ok) p.part_lse[tile.part + urow] = l > 0.f ? m + fast_log2(l) : -INFINITY;
       if (n > 0) {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar.o_free);
+        if (lane == 0) mbar_arrive(&bar.o_free[qt]);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

@@ -32,7 +32,7 @@ struct SimtCfg {
   static constexpr int ITERS = kSimtChunkKeys / KPI;
   static constexpr int CHUNK_ELEMS = kSimtChunkKeys * D;
   static constexpr int CHUNK_BYTES = CHUNK_ELEMS * 2;
-  static constexpr int NST = D == 64 ? 4 : 2;       // stages in the ring
+  static constexpr int NST = D == 64 ? 6 : 3;       // stages in the ring
   static constexpr int STAGE_ELEMS = 2 * kSimtConsumers * CHUNK_ELEMS;   // K chunks, V chunks
 };
 
@@ -76,36 +76,44 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
 
   if (warp == kSimtConsumers) {
     // ------------------------------------------------------------- producer warp
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      uint32_t use = 0;
-      for (int t = t_begin; t < t_end && !sm.abort; ++t) {
-        const Tile tile = plan.tiles[t];
-        const int nch = (tile.kv1 - tile.kv0 + kSimtChunkKeys - 1) / kSimtChunkKeys;
-        const int32_t* pages = plan.d + plan.c[tile.req];
-        for (int c0 = 0; c0 < nch; c0 += kSimtConsumers, ++use) {
-          const int s = use % C::NST;
-          if (use >= uint32_t(C::NST) && !wait_bounded(&sm.empty[s], ((use / C::NST) - 1) & 1, wc, 101))
-            break;
-          const int cnt = min(kSimtConsumers, nch - c0);
-          mbar_arrive_expect_tx(&sm.full[s], uint32_t(cnt) * 2u * C::CHUNK_BYTES);
-          for (int i = 0; i < cnt; ++i) {
-            const int key = tile.kv0 + (c0 + i) * kSimtChunkKeys;
-            const int page = pages[key / geo.page_size];
-            const int64_t row = (int64_t(page) * geo.hkv + tile.kv_head) * geo.page_size +
-                                key % geo.page_size;
-            bulk_load(&sm.stage[s][i * C::CHUNK_ELEMS], k_pool + row * D, C::CHUNK_BYTES,
-                      &sm.full[s], pol);
-            bulk_load(&sm.stage[s][(kSimtConsumers + i) * C::CHUNK_ELEMS], v_pool + row * D,
-                      C::CHUNK_BYTES, &sm.full[s], pol);
-          }
+    // Lane i issues the copies of chunk i of a stage; each lane reads its chunk's page id
+    // before the stage's empty-barrier wait, so those reads overlap it and each other.
+    const uint64_t pol = policy_evict_first();
+    uint32_t use = 0;
+    bool ok = true;
+    for (int t = t_begin; t < t_end && ok; ++t) {
+      const Tile tile = plan.tiles[t];
+      const int nch = (tile.kv1 - tile.kv0 + kSimtChunkKeys - 1) / kSimtChunkKeys;
+      const int32_t* pages = plan.d + plan.c[tile.req];
+      for (int c0 = 0; c0 < nch; c0 += kSimtConsumers, ++use) {
+        const int s = use % C::NST;
+        const int cnt = min(kSimtConsumers, nch - c0);
+        int64_t row = 0;
+        if (lane < cnt) {
+          const int key = tile.kv0 + (c0 + lane) * kSimtChunkKeys;
+          const int page = pages[key / geo.page_size];
+          row = (int64_t(page) * geo.hkv + tile.kv_head) * geo.page_size + key % geo.page_size;
+        }
+        if (lane == 0 && use >= uint32_t(C::NST))
+          ok = wait_bounded(&sm.empty[s], ((use / C::NST) - 1) & 1, wc, 101);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], uint32_t(cnt) * 2u * C::CHUNK_BYTES);
+        __syncwarp();
+        if (lane < cnt) {
+          bulk_load(&sm.stage[s][lane * C::CHUNK_ELEMS], k_pool + row * D, C::CHUNK_BYTES,
+                    &sm.full[s], pol);
+          bulk_load(&sm.stage[s][(kSimtConsumers + lane) * C::CHUNK_ELEMS], v_pool + row * D,
+                    C::CHUNK_BYTES, &sm.full[s], pol);
         }
       }
-      // Let every armed stage land before the CTA can exit (all of them when no wait gave up).
+    }
+    // Let every armed stage land before the CTA can exit (all of them when no wait gave up).
+    if (lane == 0) {
       const uint32_t armed = use;
       for (uint32_t u = armed > uint32_t(C::NST) ? armed - C::NST : 0; u < armed; ++u) {
         const int s = u % C::NST;
-        uint64_t t0 = global_timer_ns();
+        const uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(&sm.full[s], (u / C::NST) & 1) &&
                int64_t(global_timer_ns() - t0) < timeout_ns) {
         }

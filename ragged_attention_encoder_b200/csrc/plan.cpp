@@ -31,6 +31,8 @@ int64_t align4(int64_t w) { return (w + 3) & ~int64_t(3); }
 
 struct Unit {
   int32_t req, kvh, q0, qn, nkeys, rows;
+  int32_t w;       // work per key block: the number of 128-row query tiles the unit holds
+  int64_t group;   // units of one group read the same K/V (one request or span, one KV head)
 };
 
 struct Piece {
@@ -135,7 +137,7 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
   int64_t total = 0, maxc = 0;
   for (int64_t u = 0; u < nu; ++u) {
     nb[u] = ceil_div(units[u].nkeys, blk);
-    cost[u] = nb[u] + ovh;
+    cost[u] = nb[u] * units[u].w + ovh;
     total += cost[u];
     maxc = std::max(maxc, cost[u]);
   }
@@ -145,13 +147,31 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
   int32_t num_ctas = 0;
 
   auto lpt = [&]() {
-    // Longest-processing-time-first: whole units, each to the least-loaded CTA.
+    // Whole units, each to the least-loaded CTA, in an order that keeps the units sharing
+    // K/V together in time (so their K/V stay in L2) and still starts the big work first:
+    // groups by descending total cost, units within a group by descending cost.
     pieces.clear();
     std::fill(npieces.begin(), npieces.end(), 0);
     std::vector<int64_t> order(nu);
     for (int64_t u = 0; u < nu; ++u) order[u] = u;
-    std::stable_sort(order.begin(), order.end(),
-                     [&](int64_t a, int64_t b) { return cost[a] > cost[b]; });
+    std::vector<std::pair<int64_t, int64_t>> gcost;   // (group, total cost)
+    for (int64_t u = 0; u < nu; ++u) {
+      if (gcost.empty() || gcost.back().first != units[u].group) gcost.push_back({units[u].group, 0});
+      gcost.back().second += cost[u];
+    }
+    std::vector<int64_t> gtotal(nu);
+    {
+      size_t gi = 0;
+      for (int64_t u = 0; u < nu; ++u) {
+        while (gcost[gi].first != units[u].group) ++gi;
+        gtotal[u] = gcost[gi].second;
+      }
+    }
+    std::stable_sort(order.begin(), order.end(), [&](int64_t a, int64_t b) {
+      if (gtotal[a] != gtotal[b]) return gtotal[a] > gtotal[b];
+      if (units[a].group != units[b].group) return units[a].group < units[b].group;
+      return cost[a] > cost[b];
+    });
     const int32_t ctas = int32_t(std::min<int64_t>(grid, nu));
     using Load = std::pair<int64_t, int32_t>;
     std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
@@ -181,13 +201,14 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
           cap = q;
           used = false;
         }
-        const int64_t take = std::min<int64_t>(rb, std::max<int64_t>(cap - ovh, 1));
+        const int64_t w = units[u].w;
+        const int64_t take = std::min<int64_t>(rb, std::max<int64_t>((cap - ovh) / w, 1));
         if (emit) {
           pieces.push_back({int32_t(u), int32_t(s), int32_t(take), int32_t(c)});
           npieces[u] += 1;
         }
         used = true;
-        cap -= take + ovh;
+        cap -= take * w + ovh;
         s += take;
         rb -= take;
       } while (rb > 0);
@@ -361,7 +382,9 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
   for (int32_t b = 0; b < batch; ++b) max_qlen = std::max(max_qlen, qo_indptr[b + 1] - qo_indptr[b]);
   const bool simt = int64_t(max_qlen) * g <= kSimtMaxRows;
   const int32_t kind = simt ? kKindDecodeSimt : kKindTcPaged;
-  const int32_t tok_per_unit = simt ? std::max(max_qlen, 1) : kTcRows / g;
+  // tcgen05 units hold up to two 128-row query tiles that share every K/V block.
+  const int32_t tile_tok = kTcRows / g;
+  const int32_t tok_per_unit = simt ? std::max(max_qlen, 1) : 2 * tile_tok;
 
   std::vector<Unit> units;
   for (int32_t b = 0; b < batch; ++b) {
@@ -375,6 +398,8 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
         u.qn = std::min(tok_per_unit, qlen - t);
         u.nkeys = kv_len[b];
         u.rows = u.qn * g;
+        u.w = simt ? 1 : int32_t(ceil_div(u.qn, tile_tok));
+        u.group = int64_t(b) * cfg.num_kv_heads + h;
         units.push_back(u);
       }
   }
@@ -418,7 +443,8 @@ int build_ragged_plan(const rae_config& cfg, const int32_t* cu_q, const int32_t*
   if (total_q > cfg.max_q_tokens) return fail(err, RAE_ERR_CAPACITY, "total queries > max_q_tokens");
 
   const int32_t g = cfg.num_qo_heads / cfg.num_kv_heads;
-  const int32_t tok_per_unit = kTcRows / g;
+  const int32_t tile_tok = kTcRows / g;
+  const int32_t tok_per_unit = 2 * tile_tok;   // two 128-row query tiles per unit
   std::vector<Unit> units;
   for (int32_t s = 0; s < num_spans; ++s) {
     const int32_t lq = cu_q[s + 1] - cu_q[s];
@@ -437,6 +463,8 @@ int build_ragged_plan(const rae_config& cfg, const int32_t* cu_q, const int32_t*
         }
         u.nkeys = int32_t(lim);
         u.rows = u.qn * g;
+        u.w = int32_t(ceil_div(u.qn, tile_tok));
+        u.group = int64_t(s) * cfg.num_kv_heads + h;
         units.push_back(u);
       }
   }
