@@ -272,15 +272,18 @@ def _host_cfg(num_qo_heads, num_kv_heads, head_dim, page_size, num_sms, **cap):
                           cap.get("max_partial_rows", 1 << 16), num_sms)
 
 
+TILE_WORDS = 12   # {req, kv_head, q0, qn, kv0, kv1, part, split, munit, nsplit, pad, pad}
+
+
 def _decode_image(img: np.ndarray, raw: _lib.RaePlan) -> dict:
     w = img.view(np.int32)
-    n_ctas, n_tiles, n_merge = raw.num_ctas, raw.num_tiles, raw.num_merge_rows
+    n_ctas, n_tiles = raw.num_ctas, raw.num_tiles
     return {
         "header": w[:16].copy(),
         "cta_ptr": w[raw.off_cta_ptr:raw.off_cta_ptr + n_ctas + 1].copy() if n_ctas else
         np.zeros(1, np.int32),
-        "tiles": w[raw.off_tiles:raw.off_tiles + 8 * n_tiles].reshape(n_tiles, 8).copy(),
-        "merge": w[raw.off_merge:raw.off_merge + 4 * n_merge].reshape(n_merge, 4).copy(),
+        "tiles": w[raw.off_tiles:raw.off_tiles + TILE_WORDS * n_tiles].reshape(
+            n_tiles, TILE_WORDS).copy(),
         "raw": raw,
     }
 

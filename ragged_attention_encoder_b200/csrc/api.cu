@@ -40,7 +40,7 @@ struct rae_ctx {
   bool write_pending = false;
   int64_t generation = 0;
   int64_t off_slot[2] = {0, 0};
-  int64_t off_write = 0, off_part_o = 0, off_part_lse = 0, ws_bytes = 0;
+  int64_t off_write = 0, off_part_o = 0, off_part_lse = 0, off_counters = 0, ws_bytes = 0;
   int64_t timeout_ns = 4000000000LL;
   EncodeTiledFn encode = nullptr;
   std::string last_error;
@@ -78,13 +78,12 @@ DevPlan dev_plan(const rae_ctx* ctx, const rae_plan* plan, void* workspace) {
   DevPlan d;
   d.cta_ptr = img + plan->off_cta_ptr;
   d.tiles = reinterpret_cast<const Tile*>(img + plan->off_tiles);
-  d.merge = reinterpret_cast<const MergeRow*>(img + plan->off_merge);
+  d.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + ctx->off_counters);
   d.a = img + plan->off_a;
   d.b = img + plan->off_b;
   d.c = img + plan->off_c;
   d.d = img + plan->off_d;
   d.num_ctas = plan->num_ctas;
-  d.num_merge = plan->num_merge_rows;
   d.block_size = plan->block_size;
   return d;
 }
@@ -133,7 +132,8 @@ int check_plan(rae_ctx* ctx, const rae_plan* plan, bool paged) {
   if (plan->slot != 0 && plan->slot != 1) return set_err(ctx, RAE_ERR_INVALID_ARG, "bad plan slot");
   if (ctx->slot_generation[plan->slot] != plan->generation)
     return set_err(ctx, RAE_ERR_INVALID_ARG, "plan slot was re-planned since this plan was made");
-  const bool is_paged = plan->kind == kKindDecodeSimt || plan->kind == kKindTcPaged;
+  const bool is_paged = plan->kind == kKindDecodeSimt || plan->kind == kKindTcPaged ||
+                        plan->kind == kKindTcPagedSwap;
   const bool is_ragged = plan->kind == kKindTcRagged;
   if (paged ? !is_paged : !is_ragged)
     return set_err(ctx, RAE_ERR_INVALID_ARG, "plan kind does not match the run call");
@@ -155,17 +155,12 @@ float scale_log2_of(const rae_ctx* ctx, float sm_scale) {
   return s * 1.4426950408889634f;   // log2(e): scores are exponentiated with exp2
 }
 
-// Stops the attention-kernel timer, runs the merge (timed too) and closes the record.
-int finish_run(rae_ctx* ctx, const DevPlan& dp, const Geometry& geo, float* part_o,
-               float* part_lse, void* out, cudaStream_t st) {
+// Stops the attention-kernel timer and closes the record (the split-KV merge runs inside
+// the attention kernels).
+int finish_run(rae_ctx* ctx, cudaStream_t st) {
   record(timing_event(ctx, 1), st);
-  const bool has_merge = dp.num_merge > 0;
-  if (has_merge) record(timing_event(ctx, 2), st);
-  cudaError_t e = launch_merge(dp, geo, part_o, part_lse, out, st);
-  if (e != cudaSuccess) return cuda_err(ctx, e, "merge kernel launch");
-  if (has_merge) record(timing_event(ctx, 3), st);
   if (ctx->timing_count < ctx->timing_max) {
-    ctx->timing_has_merge[size_t(ctx->timing_count)] = has_merge ? 1 : 0;
+    ctx->timing_has_merge[size_t(ctx->timing_count)] = 0;
     ++ctx->timing_count;
   }
   return RAE_OK;
@@ -225,6 +220,8 @@ int rae_create(rae_ctx** out, const rae_config* cfg_in) {
   off += align256(int64_t(cfg.max_partial_rows) * cfg.head_dim * 4);
   ctx->off_part_lse = off;
   off += align256(int64_t(cfg.max_partial_rows) * 4);
+  ctx->off_counters = off;
+  off += align256(int64_t(cfg.max_tiles) * 4);
   ctx->ws_bytes = off;
 
   bool ok = true;
@@ -386,6 +383,16 @@ int rae_run_paged(rae_ctx* ctx, const rae_plan* plan, const void* q, const void*
     e = launch_decode_simt(dp, geo, q, k_pool, v_pool, out, part_o, part_lse, err, sl2,
                            ctx->timeout_ns, plan->rows_max, st);
     if (e != cudaSuccess) return cuda_err(ctx, e, "decode kernel launch");
+  } else if (plan->kind == kKindTcPagedSwap) {
+    TcTensors maps;
+    const int n_rows = plan->rows_max;
+    const int64_t rows = int64_t(num_pages) * c.num_kv_heads * c.page_size;
+    if ((rc = map_3d(ctx, &maps.q, q, c.head_dim, c.num_qo_heads, plan->total_q, geo.g, n_rows / geo.g))) return rc;
+    if ((rc = map_pool(ctx, &maps.k, k_pool, c.head_dim, rows, c.page_size))) return rc;
+    if ((rc = map_pool(ctx, &maps.v, v_pool, c.head_dim, rows, c.page_size))) return rc;
+    record(timing_event(ctx, 0), st);
+    e = launch_attn_swapab(dp, geo, n_rows, maps, out, part_o, part_lse, err, sl2, ctx->timeout_ns, st);
+    if (e != cudaSuccess) return cuda_err(ctx, e, "attention kernel launch");
   } else {
     TcTensors maps;
     const int tpt = kTcRows / geo.g;
@@ -397,7 +404,7 @@ int rae_run_paged(rae_ctx* ctx, const rae_plan* plan, const void* q, const void*
     e = launch_attn_tc(dp, geo, true, maps, out, part_o, part_lse, err, sl2, ctx->timeout_ns, st);
     if (e != cudaSuccess) return cuda_err(ctx, e, "attention kernel launch");
   }
-  return finish_run(ctx, dp, geo, part_o, part_lse, out, st);
+  return finish_run(ctx, st);
 }
 
 int rae_run_ragged(rae_ctx* ctx, const rae_plan* plan, const void* q, const void* k,
@@ -429,7 +436,7 @@ int rae_run_ragged(rae_ctx* ctx, const rae_plan* plan, const void* q, const void
   cudaError_t e = launch_attn_tc(dp, geo, false, maps, out, part_o, part_lse, err,
                                  scale_log2_of(ctx, sm_scale), ctx->timeout_ns, st);
   if (e != cudaSuccess) return cuda_err(ctx, e, "attention kernel launch");
-  return finish_run(ctx, dp, geo, part_o, part_lse, out, st);
+  return finish_run(ctx, st);
 }
 
 int rae_check_device_status(rae_ctx* ctx, void* workspace, void* stream) {
@@ -440,8 +447,11 @@ int rae_check_device_status(rae_ctx* ctx, void* workspace, void* stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_err(ctx, e, "status read");
   if (word != 0) {
-    const int zero = 0;
-    e = cudaMemcpyAsync(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice, st);
+    // A kernel that gave up may have left split arrival counters behind: clear them too.
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    e = cudaMemsetAsync(ws, 0, sizeof(int), st);
+    if (e == cudaSuccess)
+      e = cudaMemsetAsync(ws + ctx->off_counters, 0, size_t(ctx->cfg.max_tiles) * 4, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_err(ctx, e, "status clear");
     return set_err(ctx, RAE_ERR_DEVICE_TIMEOUT,

@@ -15,8 +15,8 @@
 // The MMA warp interleaves the two tiles (S0 S1 | PV0 S0' | PV1 S1' | ...) so that the tensor
 // core works on one tile while the other tile's softmax runs.  O is rescaled only when a row's
 // maximum grows by more than 2^8 (the exponent base stays stale otherwise, which is exact
-// after the final division).  The row sum l is accumulated from the bf16-rounded P that the
-// tensor core multiplies, so a constant V comes back exactly.
+// after the final division).  The row sum l adds the fp32 probabilities; the tensor core
+// multiplies their bf16 roundings.
 //
 // Warp roles (320 threads): warps 0-3 softmax + epilogue of Q0 (TMEM lanes 32w..32w+31),
 // warps 4-7 the same for Q1, warp 8 TMA producer, warp 9 MMA issuer and TMEM owner.
@@ -24,6 +24,7 @@
 // the last block are zeroed in shared memory before P.V, so junk (even NaN) in page tails
 // cannot reach the output.  Every wait is bounded.
 #include "kernels.h"
+#include "merge.cuh"
 #include "ptx.cuh"
 
 namespace rae {
@@ -35,6 +36,7 @@ constexpr int kMmaWarp = 9;
 constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kChunkBytes = 128 * 128;   // 128 rows x 64 bf16 (one 128-byte swizzle span)
+
 
 template <int D>
 struct TcLayout {
@@ -52,6 +54,8 @@ struct TcLayout {
 
 struct TcBars {
   uint64_t q_full, q_empty, fin;
+  uint64_t merge_in, merge_out;   // split-unit arrival protocol (softmax warps)
+  int merge_flag;
   uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   uint32_t tmem_base;
@@ -139,6 +143,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
     mbar_init(&bar.q_full, 1);
     mbar_init(&bar.q_empty, 1);
     mbar_init(&bar.fin, 1);
+    mbar_init(&bar.merge_in, 8);
+    mbar_init(&bar.merge_out, 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar.s_full[t], 1);
       mbar_init(&bar.p_full[t], 4);
@@ -336,13 +342,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
     const uint32_t o_col = L::o_col(qt);
     const int tok_in_tile = r / g;
     const int jh = r - tok_in_tile * g;
-    uint32_t kv_use = 0, s_cnt = 0, pv_cnt = 0;
-    for (int t = t_begin; t < t_end; ++t) {
+    uint32_t kv_use = 0, s_cnt = 0, pv_cnt = 0, split_seen = 0;
+    bool ok = true;
+    for (int t = t_begin; t < t_end && ok; ++t) {
       const Tile tile = plan.tiles[t];
       const int n = tile_blocks(tile);
       const bool has1 = tile.qn > tpt;
       if (qt == 1 && !has1) {
         kv_use += n;
+        if (tile.part >= 0 &&
+            split_unit_complete(plan.counters, tile, &bar.merge_in, &bar.merge_out, &bar.merge_flag,
+                                split_seen++, false, lane, wc, &ok))
+          merge_split_unit<D>(tile, geo, p.part_o, p.part_lse, p.out, threadIdx.x, 256);
         continue;
       }
       const int tok = qt * tpt + tok_in_tile;     // token index within the work tile
@@ -350,6 +361,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       const int q_tok = tile.q0 + tok;
       const int head = tile.kv_head * g + jh;
       const int urow = tok * g + jh;               // row within the unit (partials)
+      // A warp whose 32 rows are all padding does no softmax or epilogue work; it only keeps
+      // in step with the barriers (and zeroes stale V rows when it belongs to the first tile).
+      const bool live = __any_sync(0xffffffffu, row_ok);
       // Keys visible to this row, as a limit on the logical key index.
       int lim = tile.kv1;
       if (!p.paged) {
@@ -363,7 +377,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         lim = min(lim, rl);
       }
       float m = -INFINITY, l = 0.f;
-      bool ok = true;
       for (int j = 0; j < n; ++j) {
         const uint32_t use = kv_use + j;
         ok = __all_sync(0xffffffffu, wait_bounded(&bar.s_full[qt], s_cnt & 1, wc, 221));
@@ -372,6 +385,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         tc_fence_after();
         const int key0 = tile.kv0 + j * kTcBlockKeys;
         const int nv = max(0, min(kTcBlockKeys, lim - key0));
+        if (live) {
         // Row maximum of the raw scores with independent partial maxima (no serial chain);
         // keys past the row's limit become -inf (only in blocks that have any).
         const bool full = __all_sync(0xffffffffu, nv == kTcBlockKeys);
@@ -403,17 +417,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         const float corr = rescale ? fast_exp2(m - mn) : 1.f;
         if (need) m = mn;
         const float nbase = (m == -INFINITY) ? 0.f : -m;
-        // p = 2^(s * scale - m) rounded to bf16 and stored over the first 64 columns of S;
-        // the row sum adds exactly those bf16 values.
+        // p = 2^(s * scale - m), stored as bf16 over the first 64 columns of S; the row sum
+        // adds the fp32 values (the bf16 rounding of P is unbiased and averages out).
+        const uint64_t scale2 = f32x2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nbase2 = f32x2_pack(nbase, nbase);
         uint64_t ps[2] = {0, 0};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            pk[e] = pack_bf16x2(fast_exp2(fmaf(__uint_as_float(sv[c][2 * e]), p.scale_log2, nbase)),
-                                fast_exp2(fmaf(__uint_as_float(sv[c][2 * e + 1]), p.scale_log2, nbase)));
-            ps[e & 1] = f32x2_add(ps[e & 1], bf16x2_to_f32x2(pk[e]));
+            const uint64_t x = f32x2_fma(f32x2_pack(__uint_as_float(sv[c][2 * e]), __uint_as_float(sv[c][2 * e + 1])),
+                                         scale2, nbase2);
+            const float p0 = fast_exp2(f32x2_lo(x)), p1 = fast_exp2(f32x2_hi(x));
+            pk[e] = pack_bf16x2(p0, p1);
+            ps[e & 1] = f32x2_add(ps[e & 1], f32x2_pack(p0, p1));
           }
           tmem_st16(lane_addr + s_col + c * 16, pk);
         }
@@ -427,6 +445,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
           rescale_o<D>(lane_addr + o_col, corr);
         }
         tmem_wait_st();
+        }
         // V rows past the block's valid keys hold stale or junk data: zero them (the first
         // tile's warpgroup does it; P.V of either tile is issued after its p_full).
         const int vb = min(kTcBlockKeys, tile.kv1 - key0);
@@ -450,6 +469,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       kv_use += n;
       // ---------------------------------------------------------------- epilogue
       const bool split = tile.part >= 0;
+      if (!live) {
+        pv_cnt += n;
+      } else {
       if (n > 0) {
         ok = __all_sync(0xffffffffu, wait_bounded(&bar.pv_done[qt], (pv_cnt + n - 1) & 1, wc, 224));
         if (!ok) break;
@@ -485,11 +507,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         }
       }
       if (split && row_ok) p.part_lse[tile.part + urow] = l > 0.f ? m + fast_log2(l) : -INFINITY;
+      }
       if (n > 0) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar.o_free[qt]);
       }
+      // The CTA that completes the unit's last split merges its rows.
+      if (split &&
+          split_unit_complete(plan.counters, tile, &bar.merge_in, &bar.merge_out, &bar.merge_flag,
+                              split_seen++, threadIdx.x == 0, lane, wc, &ok))
+        merge_split_unit<D>(tile, geo, p.part_o, p.part_lse, p.out, threadIdx.x, 256);
     }
   }
 

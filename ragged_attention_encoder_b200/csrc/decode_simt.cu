@@ -17,6 +17,7 @@
 //     and the tile writes bf16 output, or an fp32 partial plus its log2-sum-exp when the
 //     plan split the unit's keys.
 #include "kernels.h"
+#include "merge.cuh"
 #include "ptx.cuh"
 
 namespace rae {
@@ -45,6 +46,8 @@ struct SimtSmem {
   float cacc[kSimtConsumers][R][D];
   uint64_t full[C::NST];
   uint64_t empty[C::NST];
+  uint64_t merge_in, merge_out;   // split-unit arrival protocol
+  int merge_flag;
   int abort;
 };
 
@@ -65,6 +68,8 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], kSimtConsumers);
     }
+    mbar_init(&sm.merge_in, kSimtConsumers);
+    mbar_init(&sm.merge_out, 1);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -125,7 +130,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
   // --------------------------------------------------------------- consumer warps
   const int grp = lane / C::CPL;   // key within a warp-wide read
   const int cl = lane % C::CPL;    // 16-byte column of the key row
-  uint32_t use = 0;
+  uint32_t use = 0, split_seen = 0;
   for (int t = t_begin; t < t_end; ++t) {
     const Tile tile = plan.tiles[t];
     const int rows = tile.qn * geo.g;
@@ -285,6 +290,15 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
           if (dc == 0) part_lse[tile.part + r] = den > 0.f ? mx + fast_log2(den) : -INFINITY;
         }
       }
+    }
+    if (tile.part >= 0) {
+      // The CTA that completes the unit's last split merges its rows.
+      bool ok = true;
+      const bool last = split_unit_complete(plan.counters, tile, &sm.merge_in, &sm.merge_out,
+                                            &sm.merge_flag, split_seen++, threadIdx.x == 0, lane,
+                                            wc, &ok);
+      if (last && !sm.abort)
+        merge_split_unit<D>(tile, geo, part_o, part_lse, out, threadIdx.x, kSimtConsumers * 32);
     }
     named_bar_sync(1, kSimtConsumers * 32);
   }

@@ -13,13 +13,12 @@ namespace rae {
 struct DevPlan {
   const int32_t* cta_ptr;   // [num_ctas + 1]
   const Tile* tiles;        // [num_tiles]
-  const MergeRow* merge;    // [num_merge]
+  int* counters;            // arrival counter per split unit (zero between runs)
   const int32_t* a;         // paged: qo_indptr   ragged: cu_q
   const int32_t* b;         // paged: kv_len      ragged: cu_kv
   const int32_t* c;         // paged: kv_page_indptr
   const int32_t* d;         // paged: kv_page_indices
   int32_t num_ctas;
-  int32_t num_merge;
   int32_t block_size;
 };
 
@@ -48,8 +47,9 @@ cudaError_t launch_attn_tc(const DevPlan& plan, const Geometry& geo, bool paged,
                            const TcTensors& maps, void* out, float* part_o, float* part_lse,
                            int* err, float scale_log2, int64_t timeout_ns, cudaStream_t stream);
 
-// Split-KV merge of partial rows into bf16 outputs.
-cudaError_t launch_merge(const DevPlan& plan, const Geometry& geo, const float* part_o,
-                         const float* part_lse, void* out, cudaStream_t stream);
+// tcgen05 attention with keys on the MMA M side, for n_rows (32 or 64) query rows, d = 128.
+cudaError_t launch_attn_swapab(const DevPlan& plan, const Geometry& geo, int n_rows,
+                               const TcTensors& maps, void* out, float* part_o, float* part_lse,
+                               int* err, float scale_log2, int64_t timeout_ns, cudaStream_t stream);
 
 }  // namespace rae

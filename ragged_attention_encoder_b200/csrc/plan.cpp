@@ -55,8 +55,7 @@ int64_t max_merge_rows(const rae_config& cfg) {
 int64_t image_bound(const rae_config& cfg) {
   int64_t w = kHdrWords;
   w = align4(w + max_ctas_for(cfg) + 1);
-  w = align4(w + int64_t(cfg.max_tiles) * 8);
-  w = align4(w + max_merge_rows(cfg) * 4);
+  w = align4(w + int64_t(cfg.max_tiles) * 12);
   w = align4(w + cfg.max_batch + 1) + align4(cfg.max_batch + 1) + align4(cfg.max_batch + 1);
   w = align4(w + cfg.max_kv_pages);
   return w;
@@ -67,7 +66,8 @@ struct Schedule {
   int32_t kind = kKindNone;
   std::vector<int32_t> cta_ptr;
   std::vector<Tile> tiles;
-  std::vector<MergeRow> merge;
+  int64_t merge_rows = 0;    // output rows merged from split partials
+  int64_t split_units = 0;   // units whose keys were split
 };
 
 // Packs a schedule and the request arrays into `image` (compact, offsets in the header).
@@ -78,9 +78,7 @@ int emit_image(const Schedule& sc, const int32_t* a, int64_t na, const int32_t* 
   const int64_t o_cta = w;
   w = align4(w + int64_t(sc.cta_ptr.size()));
   const int64_t o_tiles = w;
-  w = align4(w + int64_t(sc.tiles.size()) * 8);
-  const int64_t o_merge = w;
-  w = align4(w + int64_t(sc.merge.size()) * 4);
+  w = align4(w + int64_t(sc.tiles.size()) * 12);
   const int64_t o_a = w;
   w = align4(w + na);
   const int64_t o_b = w;
@@ -92,8 +90,7 @@ int emit_image(const Schedule& sc, const int32_t* a, int64_t na, const int32_t* 
   if (w > image_words) return fail(err, RAE_ERR_CAPACITY, "plan image exceeds its slot");
   std::memset(image, 0, size_t(w) * sizeof(int32_t));
   if (!sc.cta_ptr.empty()) std::memcpy(image + o_cta, sc.cta_ptr.data(), sc.cta_ptr.size() * 4);
-  if (!sc.tiles.empty()) std::memcpy(image + o_tiles, sc.tiles.data(), sc.tiles.size() * 32);
-  if (!sc.merge.empty()) std::memcpy(image + o_merge, sc.merge.data(), sc.merge.size() * 16);
+  if (!sc.tiles.empty()) std::memcpy(image + o_tiles, sc.tiles.data(), sc.tiles.size() * sizeof(Tile));
   if (na) std::memcpy(image + o_a, a, size_t(na) * 4);
   if (nb) std::memcpy(image + o_b, b, size_t(nb) * 4);
   if (nc) std::memcpy(image + o_c, c, size_t(nc) * 4);
@@ -102,10 +99,10 @@ int emit_image(const Schedule& sc, const int32_t* a, int64_t na, const int32_t* 
   image[kHdrKind] = sc.kind;
   image[kHdrNumTiles] = int32_t(sc.tiles.size());
   image[kHdrNumCtas] = int32_t(sc.cta_ptr.empty() ? 0 : sc.cta_ptr.size() - 1);
-  image[kHdrNumMerge] = int32_t(sc.merge.size());
+  image[kHdrNumMerge] = int32_t(sc.merge_rows);
+  image[kHdrSplitUnits] = int32_t(sc.split_units);
   image[kHdrOffCtaPtr] = int32_t(o_cta);
   image[kHdrOffTiles] = int32_t(o_tiles);
-  image[kHdrOffMerge] = int32_t(o_merge);
   image[kHdrOffA] = int32_t(o_a);
   image[kHdrOffB] = int32_t(o_b);
   image[kHdrOffC] = int32_t(o_c);
@@ -117,7 +114,7 @@ int emit_image(const Schedule& sc, const int32_t* a, int64_t na, const int32_t* 
   out->image_words = int32_t(w);
   out->off_cta_ptr = int32_t(o_cta);
   out->off_tiles = int32_t(o_tiles);
-  out->off_merge = int32_t(o_merge);
+  out->off_merge = 0;
   out->off_a = int32_t(o_a);
   out->off_b = int32_t(o_b);
   out->off_c = int32_t(o_c);
@@ -249,18 +246,20 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
                 "plan needs " + std::to_string(pieces.size()) + " tiles > max_tiles " +
                     std::to_string(cfg.max_tiles));
 
-  // Partial rows of the split units, and the merge map.
-  std::vector<int64_t> part_base(nu, -1);
-  int64_t prow = 0, nmerge = 0;
+  // Partial rows and arrival counters of the split units.
+  std::vector<int64_t> part_base(nu, -1), munit(nu, -1);
+  int64_t prow = 0, nmerge = 0, nsu = 0;
   for (int64_t u = 0; u < nu; ++u) {
     if (npieces[u] > 1) {
       part_base[u] = prow;
+      munit[u] = nsu++;
       prow += int64_t(npieces[u]) * units[u].rows;
       nmerge += units[u].rows;
     }
   }
   if (prow > cfg.max_partial_rows || nmerge > max_merge_rows(cfg))
     return fail(err, RAE_ERR_CAPACITY, "split-KV partials exceed max_partial_rows");
+  if (nsu > cfg.max_tiles) return fail(err, RAE_ERR_CAPACITY, "too many split units");
 
   sc->kind = kind;
   sc->cta_ptr.assign(size_t(num_ctas) + 1, 0);
@@ -282,26 +281,15 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
     t.part = part_base[size_t(p.unit)] < 0
                  ? -1
                  : int32_t(part_base[size_t(p.unit)] + int64_t(t.split) * un.rows);
+    t.munit = int32_t(munit[size_t(p.unit)]);
+    t.nsplit = npieces[size_t(p.unit)];
+    t.pad0 = 0;
+    t.pad1 = 0;
     sc->tiles[i] = t;
   }
   while (cur < num_ctas) sc->cta_ptr[size_t(++cur)] = int32_t(pieces.size());
-
-  sc->merge.clear();
-  sc->merge.reserve(size_t(nmerge));
-  for (int64_t u = 0; u < nu; ++u) {
-    if (part_base[size_t(u)] < 0) continue;
-    const Unit& un = units[size_t(u)];
-    for (int32_t r = 0; r < un.rows; ++r) {
-      MergeRow mr;
-      const int32_t tok = un.q0 + r / g;
-      const int32_t head = un.kvh * g + r % g;
-      mr.out_row = tok * cfg.num_qo_heads + head;
-      mr.nsplit = npieces[size_t(u)];
-      mr.part0 = int32_t(part_base[size_t(u)] + r);
-      mr.stride = un.rows;
-      sc->merge.push_back(mr);
-    }
-  }
+  sc->merge_rows = nmerge;
+  sc->split_units = nsu;
   return RAE_OK;
 }
 
@@ -380,11 +368,17 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
   const int32_t g = cfg.num_qo_heads / cfg.num_kv_heads;
   int32_t max_qlen = 0;
   for (int32_t b = 0; b < batch; ++b) max_qlen = std::max(max_qlen, qo_indptr[b + 1] - qo_indptr[b]);
-  const bool simt = int64_t(max_qlen) * g <= kSimtMaxRows;
-  const int32_t kind = simt ? kKindDecodeSimt : kKindTcPaged;
+  // Kernel family by query rows per (request, KV head): a few rows on CUDA cores (HBM bound),
+  // up to 64 rows (d = 128) with keys on the MMA's M side, otherwise 128-row query tiles.
+  const int64_t max_rows = int64_t(max_qlen) * g;
+  const bool simt = max_rows <= kSimtMaxRows;
+  const int32_t swap_n = max_rows <= 32 ? 32 : 64;
+  const bool swap = !simt && cfg.head_dim == 128 && max_rows <= 64 && swap_n % g == 0;
+  const int32_t kind = simt ? kKindDecodeSimt : (swap ? kKindTcPagedSwap : kKindTcPaged);
   // tcgen05 units hold up to two 128-row query tiles that share every K/V block.
   const int32_t tile_tok = kTcRows / g;
-  const int32_t tok_per_unit = simt ? std::max(max_qlen, 1) : 2 * tile_tok;
+  const int32_t tok_per_unit =
+      simt ? std::max(max_qlen, 1) : (swap ? swap_n / g : 2 * tile_tok);
 
   std::vector<Unit> units;
   for (int32_t b = 0; b < batch; ++b) {
@@ -398,7 +392,7 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
         u.qn = std::min(tok_per_unit, qlen - t);
         u.nkeys = kv_len[b];
         u.rows = u.qn * g;
-        u.w = simt ? 1 : int32_t(ceil_div(u.qn, tile_tok));
+        u.w = (simt || swap) ? 1 : int32_t(ceil_div(u.qn, tile_tok));
         u.group = int64_t(b) * cfg.num_kv_heads + h;
         units.push_back(u);
       }
@@ -409,6 +403,7 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
   out->block_size = 0;
   int32_t rows_max = 0;
   for (const Unit& u : units) rows_max = std::max(rows_max, u.rows);
+  if (swap) rows_max = swap_n;   // the row count the swapped kernel is instantiated for
   out->rows_max = rows_max;
   Schedule sc;
   // The decode kernel is HBM bound and short: an even split of the bytes over the grid

@@ -12,6 +12,7 @@ enum Kind : int32_t {
   kKindDecodeSimt = 1,   // paged, <= 8 query rows per (request, KV head): CUDA cores, HBM bound
   kKindTcPaged = 2,      // paged, tcgen05 tiles of 128 query rows
   kKindTcRagged = 3,     // ragged spans, tcgen05 tiles of 128 query rows
+  kKindTcPagedSwap = 4,  // paged, 9..64 query rows per unit, d = 128: keys on the MMA M side
 };
 
 // Plan image header (int32 words).
@@ -20,13 +21,13 @@ enum Hdr : int32_t {
   kHdrKind = 1,
   kHdrNumTiles = 2,
   kHdrNumCtas = 3,
-  kHdrNumMerge = 4,
+  kHdrNumMerge = 4,    // output rows merged from split partials (informational)
   kHdrBatch = 5,
   kHdrTotalQ = 6,
   kHdrBlockSize = 7,
   kHdrOffCtaPtr = 8,
   kHdrOffTiles = 9,
-  kHdrOffMerge = 10,
+  kHdrSplitUnits = 10, // units whose keys were split (arrival counters used)
   kHdrOffA = 11,   // paged: qo_indptr [B+1]        ragged: cu_q [S+1]
   kHdrOffB = 12,   // paged: kv_len [B]             ragged: cu_kv [S+1]
   kHdrOffC = 13,   // paged: kv_page_indptr [B+1]   ragged: unused
@@ -46,17 +47,11 @@ struct Tile {
   int32_t kv1;        // one past the last key of this tile
   int32_t part;       // -1: write out directly; else first partial row of this split
   int32_t split;      // split index within the unit (0 when unsplit)
+  int32_t munit;      // split unit (index of its arrival counter); -1 when unsplit
+  int32_t nsplit;     // splits of the unit (1 when unsplit)
+  int32_t pad0, pad1;
 };
-static_assert(sizeof(Tile) == 32, "tile is 8 words");
-
-// One output row produced by a split-KV merge.
-struct MergeRow {
-  int32_t out_row;    // token * Hq + head
-  int32_t nsplit;
-  int32_t part0;      // partial row of split 0
-  int32_t stride;     // distance between splits, in partial rows
-};
-static_assert(sizeof(MergeRow) == 16, "merge row is 4 words");
+static_assert(sizeof(Tile) == 48, "tile is 12 words");
 
 // Work-unit block granularity in keys: the tcgen05 kernels step 128 keys at a time, the
 // SIMT decode kernel 16 keys (one 16-row chunk of a page).
@@ -66,7 +61,7 @@ constexpr int32_t kSimtMaxRows = 8;
 constexpr int32_t kTcRows = 128;
 
 // Workspace layout: [error words | slot 0 image | slot 1 image | write staging | partial O |
-// partial lse], every region 256-byte aligned.
+// partial lse | split arrival counters], every region 256-byte aligned.
 constexpr int64_t kErrWordsBytes = 256;
 
 }  // namespace rae

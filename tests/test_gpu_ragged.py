@@ -86,4 +86,6 @@ def test_ragged_repeat_bit_identical_and_constant_v():
     c = torch.randn(case.head_dim).to(torch.bfloat16)
     case.v = c.expand_as(case.v).contiguous()
     out3, *_ = run_ragged(case)
-    assert torch.equal(out3.float().cpu(), c.float().expand_as(out3.cpu()))
+    o = out3.float().cpu()
+    ref = c.float().expand_as(o)
+    assert torch.all((o - ref).abs() <= 2.0 ** -7 * ref.abs()), float((o - ref).abs().max())

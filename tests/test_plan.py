@@ -1,7 +1,7 @@
 """Host-side tests of the C-ABI library: symbol exports and the plan builder (no GPU).
 
 The plan must cover every visible (query token, query head, key) triple exactly once, keep
-its merge map consistent with its splits, reject malformed inputs, and be deterministic.
+its split bookkeeping consistent, reject malformed inputs, and be deterministic.
 """
 import re
 import os
@@ -34,7 +34,7 @@ def _tiles_rows(tiles, g):
     """Expand tiles into (token, head, kv0, kv1, tile index)."""
     out = []
     for i, t in enumerate(tiles):
-        req, kvh, q0, qn, kv0, kv1, part, split = (int(x) for x in t)
+        req, kvh, q0, qn, kv0, kv1, part, split = (int(x) for x in t[:8])
         for r in range(qn * g):
             out.append((q0 + r // g, kvh * g + r % g, kv0, kv1, i))
     return out
@@ -50,15 +50,15 @@ def _check_cta_ptr(p):
 
 
 def _check_merge(p, g, hq):
-    """Every split unit has one merge row per row, its splits tile the unit's partial rows."""
+    """Splits of a unit tile its keys in order, share one arrival counter, count themselves,
+    and own disjoint partial rows; unsplit units write straight to the output."""
     tiles = p["tiles"]
-    merge = p["merge"]
     units = {}
     for t in tiles:
-        req, kvh, q0, qn, kv0, kv1, part, split = (int(x) for x in t)
-        units.setdefault((req, kvh, q0), []).append((split, kv0, kv1, part, qn))
-    n_rows = 0
-    seen_parts = set()
+        req, kvh, q0, qn, kv0, kv1, part, split, munit, nsplit = (int(x) for x in t[:10])
+        units.setdefault((req, kvh, q0), []).append((split, kv0, kv1, part, qn, munit, nsplit))
+    merge_rows = 0
+    seen_parts, seen_units = set(), set()
     for key, pieces in units.items():
         pieces.sort()
         assert [s for s, *_ in pieces] == list(range(len(pieces)))
@@ -66,26 +66,24 @@ def _check_merge(p, g, hq):
             assert a[2] == b[1], "splits of a unit must be contiguous in keys"
         qn = pieces[0][4]
         if len(pieces) == 1:
-            assert pieces[0][3] == -1
+            assert pieces[0][3] == -1 and pieces[0][5] == -1 and pieces[0][6] == 1
             continue
         rows = qn * g
-        n_rows += rows
-        for s, kv0, kv1, part, _ in pieces:
-            assert part >= 0
+        merge_rows += rows
+        munits = {pc[5] for pc in pieces}
+        assert len(munits) == 1 and min(munits) >= 0
+        assert not (munits & seen_units), "two units share an arrival counter"
+        seen_units |= munits
+        base = pieces[0][3]
+        for s, kv0, kv1, part, _, munit, nsplit in pieces:
+            assert nsplit == len(pieces)
+            assert part == base + s * rows
             for r in range(rows):
                 assert part + r not in seen_parts
                 seen_parts.add(part + r)
-        base = pieces[0][3]
-        req, kvh, q0 = key
-        for r in range(rows):
-            row = [m for m in merge if m[2] == base + r]
-            assert len(row) == 1
-            out_row, nsplit, part0, stride = (int(x) for x in row[0])
-            assert out_row == (q0 + r // g) * hq + kvh * g + r % g
-            assert nsplit == len(pieces) and stride == rows
-            for s, kv0, kv1, part, _ in pieces:
-                assert part == part0 - r + s * stride
-    assert n_rows == len(merge)
+    assert merge_rows == p["raw"].num_merge_rows == p["header"][4]
+    assert len(seen_units) == p["header"][10]
+    assert seen_units == set(range(len(seen_units)))
 
 
 @pytest.mark.parametrize("seed", range(6))
@@ -160,7 +158,7 @@ def test_plan_is_deterministic():
     kw = dict(num_qo_heads=32, num_kv_heads=8, head_dim=128, page_size=16)
     a = plan_paged_host(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages, **kw)
     b = plan_paged_host(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages, **kw)
-    for k in ("header", "cta_ptr", "tiles", "merge"):
+    for k in ("header", "cta_ptr", "tiles"):
         assert np.array_equal(a[k], b[k])
 
 
@@ -175,7 +173,7 @@ def test_plan_balances_the_grid():
     assert load.max() <= 1.02 * load[:-1].mean() + 2
 
 
-def test_decode_workloads_choose_the_simt_kernel():
+def test_workloads_choose_their_kernel_family():
     kinds = {}
     for i in (1, 2, 3, 5):
         c = inputs.workload(i)
@@ -183,7 +181,9 @@ def test_decode_workloads_choose_the_simt_kernel():
                             c.num_pages, num_qo_heads=c.num_qo_heads, num_kv_heads=c.num_kv_heads,
                             head_dim=c.head_dim, page_size=c.page_size)
         kinds[i] = p["raw"].kind
-    assert kinds[1] == 1 and kinds[2] == 1 and kinds[3] == 2 and kinds[5] == 2
+    # decode: CUDA-core kernel; 4 tokens x 8 heads at d=128: keys on the MMA M side;
+    # up to 512 rows: 128-row query tiles
+    assert kinds[1] == 1 and kinds[2] == 1 and kinds[3] == 2 and kinds[5] == 4
 
 
 @pytest.mark.parametrize("mutate,match", [
