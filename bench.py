@@ -57,6 +57,24 @@ def parse():
 
 # ---------------------------------------------------------------------- work accounting
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest x over all ranks (x itself outside a process group).  Every rank calls it
+    at the same point: it is one collective."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(bytes_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput of replicas: every rank processes the same bytes per step, and the
+    step takes the slowest rank's time."""
+    return bytes_per_rank_step * world / (ms_per_step * 1e-3) / 1e9
+
+
 def paged_work(case):
     """(flops, bytes) of one layer call: 4*d*Hq per visible (query, key) pair; valid K/V read
     once per KV head, plus Q and O."""
@@ -390,13 +408,10 @@ def run_ours(args):
     attn_ms, merge_ms = ctx.read_kernel_timing()
     ctx.enable_kernel_timing(0)
     ctx.check_device_status()
-    if world > 1:
-        t = torch.tensor([dev_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        dev_ms = float(t.item())
+    dev_ms = max_over_ranks(dev_ms, dev)
     ms_per_step = dev_ms / args.steps
     step_bytes = nbytes * LAYERS
-    value = step_bytes * world / (ms_per_step * 1e-3) / 1e9
+    value = job_gbs(step_bytes, world, ms_per_step)
 
     # ---------------------------------------------------------------- end to end
     q_host = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for q in qs]
@@ -423,12 +438,8 @@ def run_ours(args):
         p = e2e_step()
     t_end.record()
     torch.cuda.synchronize()
-    e2e_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = step_bytes * world / (e2e_ms / e2e_steps * 1e-3) / 1e9
+    e2e_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
+    e2e_value = job_gbs(step_bytes, world, e2e_ms / e2e_steps)
     h2d = sum(q.numel() * 2 for q in qs) + p.raw.image_words * 4
     d2h = sum(o.numel() * 2 for o in outs)
 

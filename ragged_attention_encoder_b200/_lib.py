@@ -6,6 +6,7 @@ import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librae.so")
+TEST_LIB_PATH = os.path.join(_HERE, "librae_test.so")
 
 RAE_OK = 0
 RAE_ERR_INVALID_ARG = 1
@@ -101,21 +102,38 @@ SIGNATURES = {
                                               ctypes.POINTER(i32)]),
 }
 
+# Entry points of include/rae_test_hooks.h, exported by librae_test.so only.
+TEST_SIGNATURES = {
+    "rae_test_silence_producer": (ctypes.c_int, [i32]),
+}
+
 _lib = None
+_test_lib = None
+
+
+def _open(path: str, signatures) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing; build it with `python -m ragged_attention_encoder_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in signatures.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
 
 
 def load() -> ctypes.CDLL:
     """Loads librae.so.  Raises if it has not been built: there is no fallback path."""
     global _lib
-    if _lib is not None:
-        return _lib
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(
-            f"{LIB_PATH} is missing; build it with `python -m ragged_attention_encoder_b200.build`")
-    lib = ctypes.CDLL(LIB_PATH)
-    for name, (res, args) in SIGNATURES.items():
-        fn = getattr(lib, name)
-        fn.restype = res
-        fn.argtypes = args
-    _lib = lib
-    return lib
+    if _lib is None:
+        _lib = _open(LIB_PATH, SIGNATURES)
+    return _lib
+
+
+def load_test() -> ctypes.CDLL:
+    """Loads librae_test.so (the library plus its fault-injection hooks), for tests only."""
+    global _test_lib
+    if _test_lib is None:
+        _test_lib = _open(TEST_LIB_PATH, {**SIGNATURES, **TEST_SIGNATURES})
+    return _test_lib

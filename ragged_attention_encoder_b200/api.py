@@ -103,8 +103,10 @@ class Context:
     def __init__(self, num_qo_heads: int, num_kv_heads: int, head_dim: int, page_size: int = 16, *,
                  max_batch: int = 1024, max_q_tokens: int = 1 << 17, max_kv_pages: int = 1 << 18,
                  max_tiles: int = 1 << 16, max_partial_rows: int = 1 << 16, num_sms: int = 0,
-                 device=None):
-        self._lib = _lib.load()
+                 device=None, library=None):
+        # `library`: an already loaded build of the C library (the tests pass the hooked
+        # test build); by default librae.so.
+        self._lib = library if library is not None else _lib.load()
         self.device = torch.device("cuda", torch.cuda.current_device()) if device is None \
             else torch.device(device)
         cfg = _lib.RaeConfig(num_qo_heads, num_kv_heads, head_dim, page_size, max_batch,

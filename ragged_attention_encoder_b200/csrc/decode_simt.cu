@@ -21,6 +21,13 @@
 #include "ptx.cuh"
 
 namespace rae {
+
+#ifdef RAE_TEST_HOOKS
+// Fault injection for the bounded-wait tests (test build only): the producer warp of this CTA
+// arms no copies, so the CTA's consumer waits run out.  -1: off.
+__device__ int g_silent_producer_cta = -1;
+#endif
+
 namespace {
 
 constexpr int kSimtConsumers = 4;
@@ -86,6 +93,9 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
     const uint64_t pol = policy_evict_first();
     uint32_t use = 0;
     bool ok = true;
+#ifdef RAE_TEST_HOOKS
+    if (int(blockIdx.x) == g_silent_producer_cta) ok = false;   // no copy is ever in flight
+#endif
     for (int t = t_begin; t < t_end && ok; ++t) {
       const Tile tile = plan.tiles[t];
       const int nch = (tile.kv1 - tile.kv0 + kSimtChunkKeys - 1) / kSimtChunkKeys;
@@ -351,3 +361,14 @@ cudaError_t launch_decode_simt(const DevPlan& plan, const Geometry& geo, const v
 }
 
 }  // namespace rae
+
+#ifdef RAE_TEST_HOOKS
+#include "rae_test_hooks.h"
+
+extern "C" int rae_test_silence_producer(int32_t cta) {
+  const int v = cta;
+  return cudaMemcpyToSymbol(rae::g_silent_producer_cta, &v, sizeof(int)) == cudaSuccess
+             ? RAE_OK
+             : RAE_ERR_CUDA;
+}
+#endif

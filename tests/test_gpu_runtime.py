@@ -1,9 +1,10 @@
-"""Runtime behaviour on the GPU: plan slots, staging race, stale plans and status words."""
+"""Runtime behaviour on the GPU: plan slots, staging race, stale plans, status words and the
+bounded-wait failure path."""
 import numpy as np
 import pytest
 import torch
 
-from ragged_attention_encoder_b200 import Context, inputs
+from ragged_attention_encoder_b200 import Context, RaeError, _lib, inputs
 
 from gpu_util import assert_close, gpu_pools, oracle_paged
 
@@ -81,3 +82,33 @@ def test_status_word_is_clear_after_normal_runs():
         ctx.run_paged(plan, c.q.cuda(), kp, vp)
     ctx.check_device_status()
     assert int(ctx.workspace[:4].view(torch.int32).item()) == 0
+
+
+def test_bounded_wait_runs_out_and_the_context_recovers():
+    """One CTA's producer arms nothing (test build hook): its consumers' waits run out after the
+    wait timeout, the kernel exits, the host reads RAE_ERR_DEVICE_TIMEOUT, and the same plan
+    then runs exactly (status word and split arrival counters were cleared)."""
+    lib = _lib.load_test()
+    c = _case(220)
+    ctx = Context(8, 2, 64, 16, num_sms=2, library=lib)
+    kp, vp = gpu_pools(c, ctx)
+    plan = ctx.plan_paged(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages)
+    assert plan.kernel_kind == 1 and plan.num_ctas == 4 and plan.num_merge_rows > 0
+    ref = oracle_paged(c)
+    q = c.q.cuda()
+    ctx.set_wait_timeout_ns(5_000_000)
+    assert lib.rae_test_silence_producer(1) == _lib.RAE_OK
+    try:
+        ctx.run_paged(plan, q, kp, vp)
+        with pytest.raises(RaeError) as info:
+            ctx.check_device_status()
+        assert info.value.status == _lib.RAE_ERR_DEVICE_TIMEOUT
+        assert "site 102" in str(info.value)     # a consumer's wait for a stage to fill
+    finally:
+        assert lib.rae_test_silence_producer(-1) == _lib.RAE_OK
+    ctx.set_wait_timeout_ns(4_000_000_000)
+    assert int(ctx.workspace[:4].view(torch.int32).item()) == 0
+    for _ in range(2):
+        out = ctx.run_paged(plan, q, kp, vp)
+        ctx.check_device_status()
+        assert_close(out, ref, what="after a timed-out run")

@@ -30,6 +30,18 @@ def test_library_exports_every_declared_symbol(built_library):
         assert hasattr(built_library, name), name
 
 
+def test_test_build_exports_its_hooks_and_the_product_does_not(built_library):
+    with open(os.path.join(ROOT, "include", "rae_test_hooks.h")) as f:
+        header = f.read()
+    declared = set(re.findall(r"^\s*(?:[\w\s\*]+?)\b(rae_\w+)\s*\(", header, flags=re.M))
+    assert declared == set(_lib.TEST_SIGNATURES), declared
+    test_lib = _lib.load_test()
+    for name in list(_lib.SIGNATURES) + list(declared):
+        assert hasattr(test_lib, name), name
+    for name in declared:
+        assert not hasattr(built_library, name), name
+
+
 def _tiles_rows(tiles, g):
     """Expand tiles into (token, head, kv0, kv1, tile index)."""
     out = []
