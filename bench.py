@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--skip-workloads", action="store_true",
                     help="only the headline workload (no per-workload table)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--profile-case", type=int, default=None, choices=[1, 2, 3, 4, 5],
+                    help="run only this workload's layer call --reps times (for ncu captures)")
+    ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
 
 
@@ -219,40 +222,47 @@ def time_layer_calls(ctx, calls, warmup, reps, flush_buf):
     return [a + m for a, m in zip(attn, merge)], attn, merge
 
 
+def setup_workload(i, dev):
+    """One workload's context, plan and layer call on `dev`: (case, ctx, plan, call, flops,
+    bytes, host plan µs).  Paged workloads get their context through the context write."""
+    import torch
+    from ragged_attention_encoder_b200 import Context, inputs
+    case = inputs.workload(i)
+    if hasattr(case, "kv_page_indices"):
+        ctx = Context(case.num_qo_heads, case.num_kv_heads, case.head_dim, case.page_size,
+                      device=dev)
+        kp = inputs.nan_pool(case.num_pages, case.num_kv_heads, case.page_size, case.head_dim, dev)
+        vp = inputs.nan_pool(case.num_pages, case.num_kv_heads, case.page_size, case.head_dim, dev)
+        ctx.write_context(case.k_ctx.to(dev), case.v_ctx.to(dev), case.cu_enc,
+                          case.kv_page_indptr, case.kv_page_indices, kp, vp)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        plan = ctx.plan_paged(case.qo_indptr, case.kv_page_indptr, case.kv_page_indices,
+                              case.kv_len, case.num_pages)
+        plan_us = (time.perf_counter() - t0) * 1e6
+        q = case.q.to(dev)
+        out = torch.empty_like(q)
+        call = lambda: ctx.run_paged(plan, q, kp, vp, out)  # noqa: E731
+        flops, nbytes, _ = paged_work(case)
+    else:
+        ctx = Context(case.num_qo_heads, case.num_kv_heads, case.head_dim, 16, device=dev)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        plan = ctx.plan_ragged(case.cu_q, None, case.block_size)
+        plan_us = (time.perf_counter() - t0) * 1e6
+        q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+        out = torch.empty_like(q)
+        call = lambda: ctx.run_ragged(plan, q, k, v, out)  # noqa: E731
+        flops, nbytes, _ = ragged_work(case)
+    return case, ctx, plan, call, flops, nbytes, plan_us
+
+
 def workload_table(dev, peaks, flush_buf):
     """Per-layer-call numbers of the five workloads (each one layer, L2 flushed)."""
     import torch
-    from ragged_attention_encoder_b200 import Context, inputs
     rows = {}
     for i in (1, 2, 3, 4, 5):
-        case = inputs.workload(i)
-        paged = hasattr(case, "kv_page_indices")
-        if paged:
-            ctx = Context(case.num_qo_heads, case.num_kv_heads, case.head_dim, case.page_size,
-                          device=dev)
-            kp = inputs.nan_pool(case.num_pages, case.num_kv_heads, case.page_size, case.head_dim, dev)
-            vp = inputs.nan_pool(case.num_pages, case.num_kv_heads, case.page_size, case.head_dim, dev)
-            ctx.write_context(case.k_ctx.to(dev), case.v_ctx.to(dev), case.cu_enc,
-                              case.kv_page_indptr, case.kv_page_indices, kp, vp)
-            torch.cuda.synchronize()
-            t0 = time.perf_counter()
-            plan = ctx.plan_paged(case.qo_indptr, case.kv_page_indptr, case.kv_page_indices,
-                                  case.kv_len, case.num_pages)
-            plan_us = (time.perf_counter() - t0) * 1e6
-            q = case.q.to(dev)
-            out = torch.empty_like(q)
-            call = lambda: ctx.run_paged(plan, q, kp, vp, out)  # noqa: E731
-            flops, nbytes, kvb = paged_work(case)
-        else:
-            ctx = Context(case.num_qo_heads, case.num_kv_heads, case.head_dim, 16, device=dev)
-            torch.cuda.synchronize()
-            t0 = time.perf_counter()
-            plan = ctx.plan_ragged(case.cu_q, None, case.block_size)
-            plan_us = (time.perf_counter() - t0) * 1e6
-            q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
-            out = torch.empty_like(q)
-            call = lambda: ctx.run_ragged(plan, q, k, v, out)  # noqa: E731
-            flops, nbytes, kvb = ragged_work(case)
+        case, ctx, plan, call, flops, nbytes, plan_us = setup_workload(i, dev)
         tot, attn, merge = time_layer_calls(ctx, call, 3, 20, flush_buf)
         ctx.check_device_status()
         t = statistics.median(tot) * 1e-3
@@ -556,11 +566,28 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_profile_case(args):
+    """`--profile-case I --reps N`: workload I's layer call N times and nothing else (the
+    command that ncu captures run; it prints no benchmark line)."""
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    case, ctx, plan, call, _, _, _ = setup_workload(args.profile_case, dev)
+    for _ in range(args.reps):
+        call()
+    torch.cuda.synchronize()
+    ctx.check_device_status()
+    print(json.dumps({"profile_case": case.name, "reps": args.reps, "kind": plan.kernel_kind,
+                      "tiles": plan.num_tiles, "ctas": plan.num_ctas}), flush=True)
+
+
 def main():
     args = parse()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile_case is not None:
+        run_profile_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -159,46 +159,60 @@ __global__ void __launch_bounds__(kSwThreads, 1) attn_swapab_kernel(const __grid
 
   if (warp == 4) {
     // ================================================================ TMA producer
-    if (lane == 0) {
-      const uint64_t pol_q = policy_evict_first();
-      const uint64_t pol_kv = policy_evict_first();
-      uint32_t q_use = 0, kv_use = 0;
-      bool ok = true;
-      for (int t = t_begin; t < t_end && ok && !bar.abort; ++t) {
-        const Tile tile = plan.tiles[t];
-        const int n = (tile.kv1 - tile.kv0 + kTcBlockKeys - 1) / kTcBlockKeys;
-        if (n == 0) continue;
-        if (q_use > 0 && !wait_bounded(&bar.q_empty, (q_use - 1) & 1, wc, 401)) break;
-        mbar_arrive_expect_tx(&bar.q_full, 2u * L::QCH);
-        for (int c = 0; c < 2; ++c)
-          tma_load_3d(smem + L::Q_OFF + c * L::QCH, &p.maps.q, &bar.q_full, c * 64,
-                      tile.kv_head * g, tile.q0, pol_q);
-        ++q_use;
-        const int32_t* pages = plan.d + plan.c[tile.req];
-        const int P = geo.page_size;
-        for (int j = 0; j < n; ++j, ++kv_use) {
-          const int s = kv_use % L::STAGES;
+    // The whole warp walks the tiles: lane 0 takes the barrier waits and arms the transaction
+    // counts; lane i reads the page id of the block's i-th page (before the stage's empty
+    // wait, so those reads overlap it) and issues that page's copies.
+    const uint64_t pol_q = policy_evict_first();
+    const uint64_t pol_kv = policy_evict_first();
+    uint32_t q_use = 0, kv_use = 0;
+    bool ok = true;
+    for (int t = t_begin; t < t_end && ok; ++t) {
+      const Tile tile = plan.tiles[t];
+      const int n = (tile.kv1 - tile.kv0 + kTcBlockKeys - 1) / kTcBlockKeys;
+      if (n == 0) continue;
+      if (lane == 0) {
+        if (q_use > 0 && !wait_bounded(&bar.q_empty, (q_use - 1) & 1, wc, 401)) {
+          ok = false;
+        } else {
+          mbar_arrive_expect_tx(&bar.q_full, 2u * L::QCH);
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d(smem + L::Q_OFF + c * L::QCH, &p.maps.q, &bar.q_full, c * 64,
+                        tile.kv_head * g, tile.q0, pol_q);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      ++q_use;
+      const int32_t* pages = plan.d + plan.c[tile.req];
+      const int P = geo.page_size;
+      for (int j = 0; j < n; ++j, ++kv_use) {
+        const int s = kv_use % L::STAGES;
+        const int key0 = tile.kv0 + j * kTcBlockKeys;
+        const int npg = (min(kTcBlockKeys, tile.kv1 - key0) + P - 1) / P;   // <= 8 pages
+        const uint32_t bytes = uint32_t(npg) * uint32_t(P) * 256u;
+        const int row = lane < npg ? (pages[key0 / P + lane] * geo.hkv + tile.kv_head) * P : 0;
+        if (lane == 0) {
           if (kv_use >= uint32_t(L::STAGES) &&
               !wait_bounded(&bar.kv_empty[s], ((kv_use / L::STAGES) - 1) & 1, wc, 402)) {
             ok = false;
-            break;
+          } else {
+            mbar_arrive_expect_tx(&bar.k_full[s], bytes);
+            mbar_arrive_expect_tx(&bar.v_full[s], bytes);
           }
-          const int key0 = tile.kv0 + j * kTcBlockKeys;
-          const int npg = (min(kTcBlockKeys, tile.kv1 - key0) + P - 1) / P;
-          const uint32_t bytes = uint32_t(npg) * uint32_t(P) * 256u;
-          uint8_t* ks = smem + L::K_OFF + s * kKvTile;
-          uint8_t* vs = smem + L::V_OFF + s * kKvTile;
-          mbar_arrive_expect_tx(&bar.k_full[s], bytes);
-          mbar_arrive_expect_tx(&bar.v_full[s], bytes);
-          for (int i = 0; i < npg; ++i) {
-            const int row = (pages[key0 / P + i] * geo.hkv + tile.kv_head) * P;
-            for (int c = 0; c < 2; ++c) {
-              tma_load_2d(ks + c * kChunk + i * P * 128, &p.maps.k, &bar.k_full[s], c * 64, row, pol_kv);
-              tma_load_2d(vs + c * kChunk + i * P * 128, &p.maps.v, &bar.v_full[s], c * 64, row, pol_kv);
-            }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane < npg) {
+          uint8_t* ks = smem + L::K_OFF + s * kKvTile + lane * P * 128;
+          uint8_t* vs = smem + L::V_OFF + s * kKvTile + lane * P * 128;
+          for (int c = 0; c < 2; ++c) {
+            tma_load_2d(ks + c * kChunk, &p.maps.k, &bar.k_full[s], c * 64, row, pol_kv);
+            tma_load_2d(vs + c * kChunk, &p.maps.v, &bar.v_full[s], c * 64, row, pol_kv);
           }
         }
       }
+    }
+    if (lane == 0) {
       const int64_t lim = p.timeout_ns;
       for (uint32_t u = kv_use > uint32_t(L::STAGES) ? kv_use - L::STAGES : 0; u < kv_use; ++u) {
         const int s = u % L::STAGES;

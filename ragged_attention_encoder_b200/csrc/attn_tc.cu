@@ -182,66 +182,94 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
 
   if (warp == kProducerWarp) {
     // ================================================================ TMA producer
-    if (lane == 0) {
-      const uint64_t pol_q = policy_evict_first();
-      const uint64_t pol_kv = policy_evict_last();
-      const uint32_t q_tile_bytes = uint32_t(L::CH) * 64u * 2u * uint32_t(g * tpt);
-      uint32_t q_use = 0, kv_use = 0;
-      for (int t = t_begin; t < t_end && !bar.abort; ++t) {
-        const Tile tile = plan.tiles[t];
-        const int n = tile_blocks(tile);
-        if (n == 0) continue;
-        const bool has1 = tile.qn > tpt;
-        if (q_use > 0 && !wait_bounded(&bar.q_empty, (q_use - 1) & 1, wc, 201)) break;
-        mbar_arrive_expect_tx(&bar.q_full, q_tile_bytes * (has1 ? 2u : 1u));
-        for (int qt = 0; qt < (has1 ? 2 : 1); ++qt)
+    // The whole warp walks the tiles.  Lane 0 takes the barrier waits and arms the
+    // transaction counts; for paged K/V, lane i reads the page id of the block's i-th page
+    // (before the stage's empty wait, so those reads overlap it and each other) and issues
+    // that page's copies.
+    const uint64_t pol_q = policy_evict_first();
+    const uint64_t pol_kv = policy_evict_last();
+    const uint32_t q_tile_bytes = uint32_t(L::CH) * 64u * 2u * uint32_t(g * tpt);
+    uint32_t q_use = 0, kv_use = 0;
+    bool ok = true;
+    for (int t = t_begin; t < t_end && ok; ++t) {
+      const Tile tile = plan.tiles[t];
+      const int n = tile_blocks(tile);
+      if (n == 0) continue;
+      const bool has1 = tile.qn > tpt;
+      if (lane == 0) {
+        if (q_use > 0 && !wait_bounded(&bar.q_empty, (q_use - 1) & 1, wc, 201)) {
+          ok = false;
+        } else {
+          mbar_arrive_expect_tx(&bar.q_full, q_tile_bytes * (has1 ? 2u : 1u));
+          for (int qt = 0; qt < (has1 ? 2 : 1); ++qt)
+            for (int c = 0; c < L::CH; ++c)
+              tma_load_3d(smem + L::Q_OFF + qt * L::TILE + c * kChunkBytes, &p.maps.q, &bar.q_full,
+                          c * 64, tile.kv_head * g, tile.q0 + qt * tpt, pol_q);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      ++q_use;
+      const int32_t* pages = p.paged ? plan.d + plan.c[tile.req] : nullptr;
+      const int32_t kv_base = p.paged ? 0 : plan.b[tile.req];
+      for (int j = 0; j < n; ++j, ++kv_use) {
+        const int s = kv_use % kStages;
+        const uint32_t ph = ((kv_use / kStages) - 1) & 1;
+        const int key0 = tile.kv0 + j * kTcBlockKeys;
+        uint8_t* ks = smem + L::K_OFF + s * L::TILE;
+        uint8_t* vs = smem + L::V_OFF + s * L::TILE;
+        int npg = 0, row = 0;
+        uint32_t bytes = uint32_t(L::TILE);
+        if (p.paged) {
+          const int P = geo.page_size;
+          npg = (min(kTcBlockKeys, tile.kv1 - key0) + P - 1) / P;   // <= 8 pages
+          bytes = uint32_t(npg) * uint32_t(P) * 128u * L::CH;
+          if (lane < npg) row = (pages[key0 / P + lane] * geo.hkv + tile.kv_head) * P;
+        }
+        if (lane == 0) {
+          if (kv_use >= uint32_t(kStages) && !wait_bounded(&bar.k_empty[s], ph, wc, 202)) ok = false;
+          else mbar_arrive_expect_tx(&bar.k_full[s], bytes);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (p.paged) {
+          if (lane < npg)
+            for (int c = 0; c < L::CH; ++c)
+              tma_load_2d(ks + c * kChunkBytes + lane * geo.page_size * 128, &p.maps.k, &bar.k_full[s],
+                          c * 64, row, pol_kv);
+        } else if (lane == 0) {
           for (int c = 0; c < L::CH; ++c)
-            tma_load_3d(smem + L::Q_OFF + qt * L::TILE + c * kChunkBytes, &p.maps.q, &bar.q_full,
-                        c * 64, tile.kv_head * g, tile.q0 + qt * tpt, pol_q);
-        ++q_use;
-        const int32_t* pages = p.paged ? plan.d + plan.c[tile.req] : nullptr;
-        const int32_t kv_base = p.paged ? 0 : plan.b[tile.req];
-        bool ok = true;
-        for (int j = 0; j < n; ++j, ++kv_use) {
-          const int s = kv_use % kStages;
-          const uint32_t ph = ((kv_use / kStages) - 1) & 1;
-          const int key0 = tile.kv0 + j * kTcBlockKeys;
-          uint8_t* ks = smem + L::K_OFF + s * L::TILE;
-          uint8_t* vs = smem + L::V_OFF + s * L::TILE;
-          if (kv_use >= uint32_t(kStages) && !wait_bounded(&bar.k_empty[s], ph, wc, 202)) { ok = false; break; }
-          if (p.paged) {
-            const int P = geo.page_size;
-            const int nk = min(kTcBlockKeys, tile.kv1 - key0);
-            const int npg = (nk + P - 1) / P;
-            const uint32_t bytes = uint32_t(npg) * uint32_t(P) * 128u * L::CH;
-            mbar_arrive_expect_tx(&bar.k_full[s], bytes);
-            for (int i = 0; i < npg; ++i) {
-              const int row = (pages[key0 / P + i] * geo.hkv + tile.kv_head) * P;
-              for (int c = 0; c < L::CH; ++c)
-                tma_load_2d(ks + c * kChunkBytes + i * P * 128, &p.maps.k, &bar.k_full[s], c * 64, row, pol_kv);
-            }
-            if (kv_use >= uint32_t(kStages) && !wait_bounded(&bar.v_empty[s], ph, wc, 203)) { ok = false; break; }
-            mbar_arrive_expect_tx(&bar.v_full[s], bytes);
-            for (int i = 0; i < npg; ++i) {
-              const int row = (pages[key0 / P + i] * geo.hkv + tile.kv_head) * P;
-              for (int c = 0; c < L::CH; ++c)
-                tma_load_2d(vs + c * kChunkBytes + i * P * 128, &p.maps.v, &bar.v_full[s], c * 64, row, pol_kv);
+            tma_load_3d(ks + c * kChunkBytes, &p.maps.k, &bar.k_full[s], c * 64, tile.kv_head,
+                        kv_base + key0, pol_kv);
+        }
+        if (lane == 0) {
+          if (kv_use >= uint32_t(kStages) && !wait_bounded(&bar.v_empty[s], ph, wc, 203)) {
+            ok = false;
+            // This stage's K copies are in flight: they land before the CTA may exit.
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(&bar.k_full[s], (kv_use / kStages) & 1) &&
+                   int64_t(global_timer_ns() - t0) < p.timeout_ns) {
             }
           } else {
-            mbar_arrive_expect_tx(&bar.k_full[s], uint32_t(L::TILE));
-            for (int c = 0; c < L::CH; ++c)
-              tma_load_3d(ks + c * kChunkBytes, &p.maps.k, &bar.k_full[s], c * 64, tile.kv_head,
-                          kv_base + key0, pol_kv);
-            if (kv_use >= uint32_t(kStages) && !wait_bounded(&bar.v_empty[s], ph, wc, 203)) { ok = false; break; }
-            mbar_arrive_expect_tx(&bar.v_full[s], uint32_t(L::TILE));
-            for (int c = 0; c < L::CH; ++c)
-              tma_load_3d(vs + c * kChunkBytes, &p.maps.v, &bar.v_full[s], c * 64, tile.kv_head,
-                          kv_base + key0, pol_kv);
+            mbar_arrive_expect_tx(&bar.v_full[s], bytes);
           }
         }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
+        if (p.paged) {
+          if (lane < npg)
+            for (int c = 0; c < L::CH; ++c)
+              tma_load_2d(vs + c * kChunkBytes + lane * geo.page_size * 128, &p.maps.v, &bar.v_full[s],
+                          c * 64, row, pol_kv);
+        } else if (lane == 0) {
+          for (int c = 0; c < L::CH; ++c)
+            tma_load_3d(vs + c * kChunkBytes, &p.maps.v, &bar.v_full[s], c * 64, tile.kv_head,
+                        kv_base + key0, pol_kv);
+        }
       }
-      // Drain: every armed copy lands before the CTA may exit.
+    }
+    // Drain: every armed copy lands before the CTA may exit.
+    if (lane == 0) {
       const int64_t lim = p.timeout_ns;
       for (uint32_t u = kv_use > uint32_t(kStages) ? kv_use - kStages : 0; u < kv_use; ++u) {
         const int s = u % kStages;
