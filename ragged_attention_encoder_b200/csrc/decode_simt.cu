@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
                                             &sm.merge_flag, split_seen++, threadIdx.x == 0, lane,
                                             wc, &ok);
       if (last && !sm.abort)
-        merge_split_unit<D>(tile, geo, part_o, part_lse, out, threadIdx.x, kSimtConsumers * 32);
+        merge_split_unit<D, 32 / (D / 4)>(tile, geo, part_o, part_lse, out, threadIdx.x, kSimtConsumers * 32);
     }
     named_bar_sync(1, kSimtConsumers * 32);
   }

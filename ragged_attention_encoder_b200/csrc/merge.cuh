@@ -5,8 +5,8 @@
 // O_i and lse_i = log2(sum_j 2^x_ij) (x = scaled score in log2 units).  The CTA that finishes
 // a unit's last split -- found with one arrival counter per split unit -- merges the rows:
 //     m = max_i lse_i,  w_i = 2^(lse_i - m),  O = sum_i w_i O_i / sum_i w_i
-// summed in split order (deterministic whichever CTA merges) and written as bf16.  The
-// counter is reset by that CTA, so the next run finds it at zero.
+// accumulated in split order with a running maximum (deterministic whichever CTA merges) and
+// written as bf16.  The counter is reset by that CTA, so the next run finds it at zero.
 #pragma once
 #include "kernels.h"
 #include "ptx.cuh"
@@ -46,40 +46,75 @@ __device__ __forceinline__ bool split_unit_complete(int* counters, const Tile& t
   return *flag != 0;   // partials are then read through L2 (ld.global.cg)
 }
 
-// Merges every row of the tile's unit; thread-strided over (row, 4-column group).
-template <int D>
+// Merges every row of the tile's unit.  The participating threads are whole warps
+// (tid = 32 * warp + lane, nthreads a multiple of 32).  A row's D/4 float4 column groups go to
+// consecutive lanes (one row per warp for D = 128, two for D = 64), so every partial row is
+// one coalesced read; each warp keeps kRows rows in flight (a multiple of the rows per warp
+// pass) and combines the splits in one online pass (running maximum, rescaled sums), in
+// split order.
+template <int D, int kRows>
 __device__ __forceinline__ void merge_split_unit(const Tile& tile, const Geometry& geo,
                                                  const float* part_o, const float* part_lse,
                                                  __nv_bfloat16* out, int tid, int nthreads) {
-  constexpr int V = D / 4;
+  constexpr int V = D / 4;              // float4 column groups per row
+  constexpr int RPW = 32 / V;           // rows per warp and pass
+  constexpr int U = kRows / RPW;        // passes unrolled
+  static_assert(U >= 1 && U * RPW == kRows, "kRows must be a multiple of the rows per pass");
   const int rows = tile.qn * geo.g;
   const int base = tile.part - tile.split * rows;
-  for (int e = tid; e < rows * V; e += nthreads) {
-    const int r = e / V;
-    const int c = e - r * V;
-    float m = -INFINITY;
-    for (int s = 0; s < tile.nsplit; ++s) m = fmaxf(m, __ldcg(part_lse + base + s * rows + r));
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float den = 0.f;
-    if (m != -INFINITY) {
-      for (int s = 0; s < tile.nsplit; ++s) {
-        const int row = base + s * rows + r;
-        const float w = fast_exp2(__ldcg(part_lse + row) - m);
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(part_o + int64_t(row) * D) + c);
-        den += w;
-        acc.x += w * v.x;
-        acc.y += w * v.y;
-        acc.z += w * v.z;
-        acc.w += w * v.w;
+  const int ns = tile.nsplit;
+  const int lane = tid & 31;
+  const int c = lane % V;
+  const int rsub = lane / V;
+  for (int r0 = (tid >> 5) * kRows; r0 < rows; r0 += (nthreads >> 5) * kRows) {
+    float m[U], den[U];
+    float4 acc[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      m[u] = -INFINITY;
+      den[u] = 0.f;
+      acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int s = 0; s < ns; ++s) {
+      float l[U];
+      float4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int r = r0 + u * RPW + rsub;
+        l[u] = -INFINITY;
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < rows) {
+          const int row = base + s * rows + r;
+          l[u] = __ldcg(part_lse + row);
+          v[u] = __ldcg(reinterpret_cast<const float4*>(part_o + int64_t(row) * D) + c);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (l[u] == -INFINITY) continue;             // this split saw no key of the row
+        const float mn = fmaxf(m[u], l[u]);
+        const float a = fast_exp2(m[u] - mn);         // 0 while m is still -inf
+        const float b = fast_exp2(l[u] - mn);
+        acc[u].x = acc[u].x * a + v[u].x * b;
+        acc[u].y = acc[u].y * a + v[u].y * b;
+        acc[u].z = acc[u].z * a + v[u].z * b;
+        acc[u].w = acc[u].w * a + v[u].w * b;
+        den[u] = den[u] * a + b;
+        m[u] = mn;
       }
     }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    const int tok = tile.q0 + r / geo.g;
-    const int head = tile.kv_head * geo.g + r % geo.g;
-    uint2 pk;
-    pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2*>(out + (int64_t(tok) * geo.hq + head) * D + 4 * c) = pk;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int r = r0 + u * RPW + rsub;
+      if (r >= rows) continue;
+      const float inv = den[u] > 0.f ? 1.f / den[u] : 0.f;
+      const int tok = tile.q0 + r / geo.g;
+      const int head = tile.kv_head * geo.g + r % geo.g;
+      uint2 pk;
+      pk.x = pack_bf16x2(acc[u].x * inv, acc[u].y * inv);
+      pk.y = pack_bf16x2(acc[u].z * inv, acc[u].w * inv);
+      *reinterpret_cast<uint2*>(out + (int64_t(tok) * geo.hq + head) * D + 4 * c) = pk;
+    }
   }
 }
 
