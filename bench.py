@@ -258,12 +258,13 @@ def setup_workload(i, dev):
 
 
 def workload_table(dev, peaks, flush_buf):
-    """Per-layer-call numbers of the five workloads (each one layer, L2 flushed)."""
+    """Per-layer-call numbers of the five workloads: median of 100 calls after 10 warm-up
+    calls, L2 flushed (a 256 MB write, over twice the L2) before every call."""
     import torch
     rows = {}
     for i in (1, 2, 3, 4, 5):
         case, ctx, plan, call, flops, nbytes, plan_us = setup_workload(i, dev)
-        tot, attn, merge = time_layer_calls(ctx, call, 3, 20, flush_buf)
+        tot, attn, merge = time_layer_calls(ctx, call, 10, 100, flush_buf)
         ctx.check_device_status()
         t = statistics.median(tot) * 1e-3
         ta = statistics.median(attn) * 1e-3
@@ -282,6 +283,9 @@ def workload_table(dev, peaks, flush_buf):
             "roofline_frac_of_spec": round(t_star_spec / t, 4),
             "roofline_frac_of_measured": round(t_star_meas / t, 4),
             "tc_frac_of_spec": round(tc / SPEC_TC_TFLOPS, 4),
+            "tc_frac_of_measured": round(tc / peaks["tflops"], 4),
+            "tc_frac_of_measured_sustained": round(tc / peaks["tflops_sustained"], 4),
+            "hbm_frac_of_measured": round(gbs / peaks["hbm_gbs"], 4),
             "hbm_frac_of_spec": round(gbs / SPEC_HBM_GBS, 4),
             "algorithmic_flops": flops,
             "algorithmic_bytes": nbytes,

@@ -112,3 +112,35 @@ def test_bounded_wait_runs_out_and_the_context_recovers():
         out = ctx.run_paged(plan, q, kp, vp)
         ctx.check_device_status()
         assert_close(out, ref, what="after a timed-out run")
+
+
+@pytest.mark.parametrize("qmax", [1, 40])
+def test_planned_run_calls_replay_from_a_cuda_graph(qmax):
+    """Once planned, a run call is a stream-ordered launch and nothing else: a CUDA graph that
+    captures several layer calls (decode kernel for one-token queries, the tensor-core kernel
+    for packs of up to 40) replays them with outputs bit-identical to eager calls."""
+    c = _case(230 + qmax, qmax=qmax)
+    ctx = Context(8, 2, 64, 16)
+    kp, vp = gpu_pools(c, ctx)
+    plan = ctx.plan_paged(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages)
+    assert plan.kernel_kind == (1 if qmax == 1 else 2)
+    gen = torch.Generator(device="cuda").manual_seed(qmax)
+    layers = 4
+    qs = [c.q.cuda()] + [torch.randn(c.q.shape, generator=gen, device="cuda").to(torch.bfloat16)
+                         for _ in range(layers - 1)]
+    eager = [ctx.run_paged(plan, q, kp, vp) for q in qs]
+    outs = [torch.empty_like(q) for q in qs]
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for q, o in zip(qs, outs):
+            ctx.run_paged(plan, q, kp, vp, o)
+    for o in outs:
+        o.zero_()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    ctx.check_device_status()
+    for e, o in zip(eager, outs):
+        assert torch.equal(e, o)
+    assert_close(outs[0], oracle_paged(c), what="graph replay")
