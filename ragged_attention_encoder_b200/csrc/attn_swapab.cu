@@ -152,6 +152,8 @@ __global__ void __launch_bounds__(kSwThreads, 1) attn_swapab_kernel(const __grid
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();
+  griddep_launch_dependents();
   const uint32_t tmem = bar.tmem_base;
   const WaitCtl wc{&bar.abort, p.err, p.timeout_ns};
   const int t_begin = plan.cta_ptr[blockIdx.x];
@@ -496,8 +498,8 @@ cudaError_t launch_n(const SwParams& prm, int num_ctas, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(attn_swapab_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SwLayout<N>::SMEM);
   if (e != cudaSuccess) return e;
-  attn_swapab_kernel<N><<<dim3(uint32_t(num_ctas)), kSwThreads, SwLayout<N>::SMEM, stream>>>(prm);
-  return cudaGetLastError();
+  return launch_pdl(attn_swapab_kernel<N>, dim3(uint32_t(num_ctas)), dim3(kSwThreads),
+                    SwLayout<N>::SMEM, stream, prm);
 }
 
 }  // namespace

@@ -172,6 +172,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();
+  griddep_launch_dependents();
   const uint32_t tmem = bar.tmem_base;
   const WaitCtl wc{&bar.abort, p.err, p.timeout_ns};
 
@@ -579,14 +581,16 @@ cudaError_t launch_attn_tc(const DevPlan& plan, const Geometry& geo, bool paged,
     e = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              TcLayout<128>::SMEM);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<128><<<dim3(uint32_t(plan.num_ctas)), kTcThreads, TcLayout<128>::SMEM, stream>>>(prm);
+    e = launch_pdl(attn_tc_kernel<128>, dim3(uint32_t(plan.num_ctas)), dim3(kTcThreads),
+                   TcLayout<128>::SMEM, stream, prm);
   } else {
     e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              TcLayout<64>::SMEM);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<64><<<dim3(uint32_t(plan.num_ctas)), kTcThreads, TcLayout<64>::SMEM, stream>>>(prm);
+    e = launch_pdl(attn_tc_kernel<64>, dim3(uint32_t(plan.num_ctas)), dim3(kTcThreads),
+                   TcLayout<64>::SMEM, stream, prm);
   }
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace rae

@@ -81,6 +81,8 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
     fence_mbar_init();
   }
   __syncthreads();
+  griddep_wait();
+  griddep_launch_dependents();
   const WaitCtl wc{&sm.abort, err, timeout_ns};
 
   const int t_begin = plan.cta_ptr[blockIdx.x];
@@ -326,11 +328,11 @@ cudaError_t launch_t(const DevPlan& plan, const Geometry& geo, const void* q, co
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<dim3(uint32_t(plan.num_ctas)), kSimtThreads, smem, stream>>>(
-      plan, geo, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_pool),
-      static_cast<const __nv_bfloat16*>(v_pool), static_cast<__nv_bfloat16*>(out), part_o,
-      part_lse, err, scale_log2, timeout_ns);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(uint32_t(plan.num_ctas)), dim3(kSimtThreads), smem, stream, plan,
+                    geo, static_cast<const __nv_bfloat16*>(q),
+                    static_cast<const __nv_bfloat16*>(k_pool),
+                    static_cast<const __nv_bfloat16*>(v_pool), static_cast<__nv_bfloat16*>(out),
+                    part_o, part_lse, err, scale_log2, timeout_ns);
 }
 
 template <int D>

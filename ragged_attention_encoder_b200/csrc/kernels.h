@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "plan.h"
 #include "rae_internal.h"
 
@@ -21,6 +23,25 @@ struct DevPlan {
   int32_t num_ctas;
   int32_t block_size;
 };
+
+// Launches `kern` on `stream` with programmatic stream serialisation allowed: the kernel may
+// be scheduled before the preceding kernel on the stream has finished (its prologue overlaps
+// that kernel's tail) and calls griddep_wait before its first read of global memory.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = smem;
+  lc.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, kern, std::forward<Args>(args)...);
+}
 
 struct Geometry {
   int32_t hq, hkv, g, d, page_size;
