@@ -147,6 +147,35 @@ def test_swapped_kernel_with_forced_splits(num_sms):
     assert_close(out, oracle_paged(case), what=f"swap split {num_sms}")
 
 
+@pytest.mark.parametrize("hq,hkv,d,qlens,kind", [
+    (8, 1, 128, [1, 1], 1),    # 8 rows per (request, KV head): CUDA-core decode kernel
+    (8, 1, 128, [2, 1], 4),    # 16 rows: keys on the MMA M side, 32 columns
+    (8, 1, 128, [8, 3], 4),    # 64 rows: keys on the MMA M side, 64 columns
+    (8, 1, 128, [9, 2], 2),    # 72 rows: 128-row query tiles
+    (8, 1, 64, [2, 1], 2),     # d = 64: no swapped kernel, 128-row query tiles
+])
+def test_kernel_choice_at_row_boundaries(hq, hkv, d, qlens, kind):
+    case = inputs.paged_case(190 + sum(qlens) + d, q_lens=qlens, ctx_lens=(300, 2500, len(qlens)),
+                             num_qo_heads=hq, num_kv_heads=hkv, head_dim=d, page_size=16)
+    out, plan, *_ = run_paged(case)
+    assert plan.kernel_kind == kind
+    assert_close(out, oracle_paged(case), what=f"rows boundary {qlens} d={d}")
+
+
+@pytest.mark.parametrize("qlens,hq,hkv,d,kind", [([0, 1, 0, 1, 0], 20, 20, 64, 1),
+                                                 ([0, 4, 0, 2], 64, 8, 128, 4),
+                                                 ([0, 37, 0, 5, 0], 32, 8, 128, 2)])
+def test_requests_without_queries_between_others(qlens, hq, hkv, d, kind):
+    """Requests with no query tokens (their context still in the pool) write nothing and do
+    not disturb their neighbours, in every kernel family."""
+    case = inputs.paged_case(200 + sum(qlens), q_lens=qlens, ctx_lens=(100, 2000, len(qlens)),
+                             num_qo_heads=hq, num_kv_heads=hkv, head_dim=d, page_size=16)
+    out, plan, *_ = run_paged(case)
+    assert plan.kernel_kind == kind
+    assert out.shape[0] == sum(qlens)
+    assert_close(out, oracle_paged(case), what=f"empty queries {qlens}")
+
+
 def test_empty_context_gives_zero():
     case = inputs.paged_case(61, q_lens=[2, 1, 3], ctx_lens=[0, 5, 0], num_qo_heads=4,
                              num_kv_heads=2, head_dim=64, page_size=16, pool_pages=4)
