@@ -5,6 +5,8 @@
 // One CTA copies one page's worth of tokens for K and for V.  The source rows of a page are
 // one contiguous block of ntok * Hkv * d elements, the destination is the page's Hkv runs of
 // ntok * d elements, so both sides move in whole 16-byte vectors with coalesced accesses.
+// Each thread issues four iterations' loads before their stores (eight 16-byte loads in
+// flight), and both sides stream past L2 (neither is read again soon).
 // HBM bound: algorithmic bytes = 2 (K and V) x 2 (read + write) x tokens x Hkv x d x 2 B.
 #include <mutex>
 #include <string>
@@ -27,16 +29,30 @@ __global__ void __launch_bounds__(256) context_write_kernel(const WriteItem* __r
   const int32_t n = it.ntok * per_tok;
   const int64_t src0 = int64_t(it.src_row) * per_tok;
   const int64_t page0 = int64_t(it.page) * hkv * page_size * vec_per_row;
-  for (int32_t e = threadIdx.x; e < n; e += blockDim.x) {
-    const int32_t slot = e / per_tok;
-    const int32_t rem = e - slot * per_tok;
-    const int32_t h = rem / vec_per_row;
-    const int32_t u = rem - h * vec_per_row;
-    const int64_t dst = page0 + (int64_t(h) * page_size + slot) * vec_per_row + u;
-    const uint4 kv = __ldcs(k_src + src0 + e);   // streamed once
-    const uint4 vv = __ldcs(v_src + src0 + e);
-    k_pool[dst] = kv;
-    v_pool[dst] = vv;
+  constexpr int U = 4;
+  for (int32_t e0 = threadIdx.x; e0 < n; e0 += U * blockDim.x) {
+    uint4 kv[U], vv[U];
+#pragma unroll
+    for (int i = 0; i < U; ++i) {
+      const int32_t e = e0 + i * int32_t(blockDim.x);
+      if (e < n) {
+        kv[i] = __ldcs(k_src + src0 + e);
+        vv[i] = __ldcs(v_src + src0 + e);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < U; ++i) {
+      const int32_t e = e0 + i * int32_t(blockDim.x);
+      if (e < n) {
+        const int32_t slot = e / per_tok;
+        const int32_t rem = e - slot * per_tok;
+        const int32_t h = rem / vec_per_row;
+        const int32_t u = rem - h * vec_per_row;
+        const int64_t dst = page0 + (int64_t(h) * page_size + slot) * vec_per_row + u;
+        __stcs(k_pool + dst, kv[i]);
+        __stcs(v_pool + dst, vv[i]);
+      }
+    }
   }
 }
 
