@@ -95,7 +95,7 @@ typedef struct rae_plan {
   int64_t generation;        /* increments per plan on a context */
   int32_t off_cta_ptr;       /* word offsets of the image's arrays (internal) */
   int32_t off_tiles;
-  int32_t off_merge;
+  int32_t off_merge;         /* unused, 0: the split merge is fused into the attention kernels */
   int32_t off_a;
   int32_t off_b;
   int32_t off_c;
@@ -163,9 +163,10 @@ int rae_write_context_noalloc(const void* k_src, const void* v_src, const int32_
  * Host int32 arrays: qo_indptr [B+1] (cumulative query lengths, qo_indptr[0] == 0),
  * kv_page_indptr [B+1], kv_page_indices [kv_page_indptr[B]], kv_len [B] (context tokens of
  * each request; request b needs kv_page_indptr[b+1] - kv_page_indptr[b] >= ceil(kv_len[b]/P),
- * extra pages are never read).  Validates, builds the work tiles, the split-KV schedule and
- * the merge map, stages them in slot `slot` (0 or 1) and copies them into the workspace on
- * `stream`.  *out describes the plan.
+ * extra pages are never read).  Validates, builds the work tiles and the split-KV schedule
+ * (partial rows and an arrival counter for every unit whose keys are split), stages them in
+ * slot `slot` (0 or 1) and copies them into the workspace on `stream`.  *out describes the
+ * plan.
  */
 int rae_plan_paged(rae_ctx* ctx, int32_t slot, const int32_t* qo_indptr,
                    const int32_t* kv_page_indptr, const int32_t* kv_page_indices,
@@ -207,11 +208,12 @@ int rae_set_wait_timeout_ns(rae_ctx* ctx, int64_t timeout_ns);
 
 /*
  * Kernel timing (instrumentation for measurement).  With max_records > 0, every run call
- * records CUDA events on its stream immediately before and after its attention kernel and
- * around its split-KV merge kernel, for up to max_records calls; max_records == 0 turns it off.
- * rae_read_kernel_timing synchronises those events, writes the elapsed milliseconds of each
- * recorded call to attn_ms[i] and merge_ms[i] (0 when the call had no merge), sets *count, and
- * clears the records.  Timing adds no work to the kernels themselves.
+ * records CUDA events on its stream immediately before and after its attention kernel, for up
+ * to max_records calls; max_records == 0 turns it off.  rae_read_kernel_timing synchronises
+ * those events, writes the elapsed milliseconds of each recorded call to attn_ms[i] (the split
+ * merge runs inside that kernel, so merge_ms[i] is 0), sets *count, and clears the records.
+ * Timing adds no work to the kernels, but an event between two kernels serialises their
+ * launches: time whole sequences without it.
  */
 int rae_enable_kernel_timing(rae_ctx* ctx, int32_t max_records);
 int rae_read_kernel_timing(rae_ctx* ctx, float* attn_ms, float* merge_ms, int32_t max,
@@ -222,12 +224,12 @@ int rae_read_kernel_timing(rae_ctx* ctx, float* attn_ms, float* merge_ms, int32_
  * rae_plan_paged / rae_plan_ragged, written into a caller-provided host buffer `image` of
  * image_bytes >= rae_plan_image_bytes bytes, with no CUDA call.  cfg->num_sms must be > 0.
  * The image is int32 words: a 16-word header (magic, kind, num_tiles, num_ctas,
- * num_merge_rows, batch, total_q, block_size, then word offsets of the CTA pointer array,
- * the tiles, the merge rows and the four request arrays, then the largest rows per unit)
- * followed by those arrays, packed; out->image_words words are used.
- * Tiles are 8 words {request, kv_head, first query token, query tokens, first key,
- * end key, first partial row or -1, split index}; merge rows are 4 words {token*Hq+head,
- * number of splits, partial row of split 0, partial-row stride between splits}.
+ * num_merge_rows, batch, total_q, block_size, word offsets of the CTA pointer array and of
+ * the tiles, the number of split units, word offsets of the four request arrays, the largest
+ * rows per unit) followed by those arrays, packed; out->image_words words are used.
+ * Tiles are 12 words {request, kv_head, first query token, query tokens, first key, end key,
+ * first partial row or -1, split index, arrival counter of the split unit or -1, number of
+ * splits of the unit, 0, 0}.
  */
 int rae_plan_paged_host(const rae_config* cfg, const int32_t* qo_indptr,
                         const int32_t* kv_page_indptr, const int32_t* kv_page_indices,
