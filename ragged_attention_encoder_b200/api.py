@@ -160,7 +160,8 @@ class Context:
         self._check(self._lib.rae_enable_kernel_timing(self._h, int(max_records)))
 
     def read_kernel_timing(self):
-        """(attention-kernel ms, merge-kernel ms) of each run recorded since the last read."""
+        """(attention-kernel ms, merge ms) of each run recorded since the last read; the split
+        merge runs inside the attention kernel, so the second list holds zeros."""
         n_max = 1 << 16
         a = (ctypes.c_float * n_max)()
         m = (ctypes.c_float * n_max)()
