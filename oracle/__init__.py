@@ -15,13 +15,17 @@ routine (closed forms, invariants, brute-force enumeration, and
 "parity unpinned".
 """
 from .attention import (  # noqa: F401
+    append_kv,
     as_f64,
     attention_rows,
     block_causal_visible,
     block_causal_key_limit,
+    causal_append_visible,
     context_write,
     gather_paged_kv,
     merge_partials,
+    paged_causal_attention,
+    paged_causal_attention_rows,
     paged_cross_attention,
     paged_cross_attention_rows,
     partial_attention_with_lse,

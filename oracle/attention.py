@@ -27,6 +27,11 @@ Visibility per path:
   ``block_size``; position ``i`` sees ``j`` iff ``j // bs <= i // bs``.
 * Ragged two-span cross-attention (same page, ``RaggedCrossAttnManager``): the query
   span of request ``r`` sees every key of the request's key span, non-causally.
+* Paged causal self-attention (mstar.engine.resources.attn.config, ``AttentionStep`` with
+  ``causal=True``): the step's ``qlen`` queries are the last tokens of the request's
+  ``kv_len``-token stream (their own K/V already appended); query ``i`` (0-based within the
+  step) is token ``kv_len - qlen + i`` of the stream and sees keys ``0 .. kv_len - qlen + i``.
+  The pages give only the flag; this position rule is the reading taken.
 
 The inputs are exact bf16 values; they are upcast to float64 here, so the only error in
 this module is float64 rounding.  Nothing here is blocked, fused or reordered.
@@ -167,6 +172,36 @@ def context_write(k_src: torch.Tensor, v_src: torch.Tensor, cu_enc, page_indptr,
     return k_out, v_out
 
 
+def append_kv(k_new: torch.Tensor, v_new: torch.Tensor, append_indptr, page_indptr,
+              page_indices, kv_len, k_pool: torch.Tensor, v_pool: torch.Tensor):
+    """Append of a step's own K/V to its stream, done by plain element copies (bit exact).
+
+    The n = append_indptr[b+1] - append_indptr[b] new tokens of request b (rows
+    ``append_indptr[b] + t`` of ``[sum_new, Hkv, d]``) are stream positions
+    ``kv_len[b] - n + t`` (``kv_len`` counts the tokens after the append): page
+    ``page_indices[page_indptr[b] + pos // P]``, slot ``pos % P``.  Returns new pools.
+    """
+    k_out = k_pool.clone()
+    v_out = v_pool.clone()
+    page_size = k_pool.shape[2]
+    for b in range(len(append_indptr) - 1):
+        n = int(append_indptr[b + 1]) - int(append_indptr[b])
+        for t in range(n):
+            pos = int(kv_len[b]) - n + t
+            page = int(page_indices[int(page_indptr[b]) + pos // page_size])
+            k_out[page, :, pos % page_size, :] = k_new[int(append_indptr[b]) + t]
+            v_out[page, :, pos % page_size, :] = v_new[int(append_indptr[b]) + t]
+    return k_out, v_out
+
+
+def causal_append_visible(qlen: int, kv_len: int) -> np.ndarray:
+    """[qlen, kv_len] boolean mask: query i (stream token kv_len - qlen + i) sees key j iff
+    j <= kv_len - qlen + i."""
+    i = np.arange(qlen)[:, None]
+    j = np.arange(kv_len)[None, :]
+    return j <= kv_len - qlen + i
+
+
 def _kv_head(h: int, num_qo_heads: int, num_kv_heads: int) -> int:
     return h // (num_qo_heads // num_kv_heads)
 
@@ -212,6 +247,53 @@ def paged_cross_attention_rows(q, k_pool, v_pool, qo_indptr, page_indptr, page_i
         kvh = _kv_head(h, hq, hkv)
         qrow = as_f64(q[t, h])[None, :]
         out[n] = attention_rows(qrow, kb[:, kvh], vb[:, kvh], s)[0]
+    return out
+
+
+def paged_causal_attention(q, k_pool, v_pool, qo_indptr, page_indptr, page_indices, kv_len,
+                           scale=None) -> np.ndarray:
+    """Paged causal self-attention of each request's step queries over its stream.
+
+    q [sum_q, Hq, d]; pools [num_pages, Hkv, P, d] holding each request's kv_len tokens;
+    returns float64 [sum_q, Hq, d].
+    """
+    qf = as_f64(q)
+    hq, d = qf.shape[1], qf.shape[2]
+    hkv = k_pool.shape[1]
+    s = _default_scale(d, scale)
+    out = np.zeros_like(qf)
+    for b in range(len(kv_len)):
+        q0, q1 = int(qo_indptr[b]), int(qo_indptr[b + 1])
+        if q1 == q0:
+            continue
+        kb = gather_paged_kv(k_pool, page_indptr, page_indices, b, int(kv_len[b]))
+        vb = gather_paged_kv(v_pool, page_indptr, page_indices, b, int(kv_len[b]))
+        vis = causal_append_visible(q1 - q0, int(kv_len[b]))
+        for h in range(hq):
+            kvh = _kv_head(h, hq, hkv)
+            out[q0:q1, h] = attention_rows(qf[q0:q1, h], kb[:, kvh], vb[:, kvh], s, vis)
+    return out
+
+
+def paged_causal_attention_rows(q, k_pool, v_pool, qo_indptr, page_indptr, page_indices,
+                                kv_len, rows, scale=None) -> np.ndarray:
+    """The same as ``paged_causal_attention`` for selected (token, head) pairs only."""
+    qo_indptr = np.asarray(qo_indptr)
+    d = q.shape[2]
+    hq, hkv = q.shape[1], k_pool.shape[1]
+    s = _default_scale(d, scale)
+    cache = {}
+    out = np.zeros((len(rows), d))
+    for n, (t, h) in enumerate(rows):
+        b = int(np.searchsorted(qo_indptr, t, side="right") - 1)
+        if b not in cache:
+            cache[b] = (gather_paged_kv(k_pool, page_indptr, page_indices, b, int(kv_len[b])),
+                        gather_paged_kv(v_pool, page_indptr, page_indices, b, int(kv_len[b])))
+        kb, vb = cache[b]
+        qlen = int(qo_indptr[b + 1]) - int(qo_indptr[b])
+        vis = causal_append_visible(qlen, int(kv_len[b]))[t - int(qo_indptr[b])][None, :]
+        out[n] = attention_rows(as_f64(q[t, h])[None, :], kb[:, _kv_head(h, hq, hkv)],
+                                vb[:, _kv_head(h, hq, hkv)], s, vis)[0]
     return out
 
 

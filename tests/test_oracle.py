@@ -342,3 +342,123 @@ def test_tiny_workload_oracle_golden():
                                        case.kv_page_indices, case.kv_len)
     assert np.allclose(out, np.array(g["out"]), atol=1e-12, rtol=0)
     assert math.isclose(float(np.abs(out).sum()), g["abs_sum"], rel_tol=1e-12)
+
+
+# ---------------------------------------------- paged causal self-attention and the append
+
+def _causal_case(seed, qlens, kvlens, hq=4, hkv=2, d=16, page_size=16, pool_pages=None):
+    case = inputs.paged_case(seed, q_lens=qlens, ctx_lens=kvlens, num_qo_heads=hq,
+                             num_kv_heads=hkv, head_dim=d, page_size=page_size,
+                             pool_pages=pool_pages)
+    kp, vp = _oracle_pools(case)
+    return case, kp, vp
+
+
+def _causal(case, kp, vp):
+    return oracle.paged_causal_attention(case.q, kp, vp, case.qo_indptr, case.kv_page_indptr,
+                                         case.kv_page_indices, case.kv_len)
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (4, 2), (6, 1)])
+def test_paged_causal_prefill_is_sdpa_causal(hq, hkv):
+    """A step whose queries are its whole stream (qlen == kv_len) is ordinary causal
+    self-attention over the stream, which torch computes with is_causal=True."""
+    lens = [1, 9, 33]
+    case, kp, vp = _causal_case(40 + hq, lens, lens, hq, hkv)
+    out = _causal(case, kp, vp)
+    qf, kf, vf = (oracle.as_f64(t) for t in (case.q, case.k_ctx, case.v_ctx))
+    for b in range(case.batch):
+        q0, q1 = case.qo_indptr[b], case.qo_indptr[b + 1]
+        c0, c1 = case.cu_enc[b], case.cu_enc[b + 1]
+        qt = torch.from_numpy(qf[q0:q1]).permute(1, 0, 2)[None]
+        kt = torch.from_numpy(kf[c0:c1]).permute(1, 0, 2)[None]
+        vt = torch.from_numpy(vf[c0:c1]).permute(1, 0, 2)[None]
+        ref = F.scaled_dot_product_attention(qt, kt, vt, is_causal=True,
+                                             enable_gqa=hq != hkv)[0].permute(1, 0, 2).numpy()
+        assert np.allclose(out[q0:q1], ref, atol=1e-12, rtol=0)
+
+
+def test_paged_causal_query_sees_the_stream_up_to_itself():
+    """Query i of a step is the stream's token kv_len - qlen + i: its result equals
+    cross-attention (pinned to SDPA) of that query over the stream cut just after it."""
+    case, kp, vp = _causal_case(44, [3, 1, 7, 5], [20, 5, 40, 5])
+    out = _causal(case, kp, vp)
+    for b in range(case.batch):
+        q0, q1 = int(case.qo_indptr[b]), int(case.qo_indptr[b + 1])
+        qlen, kvl = q1 - q0, int(case.kv_len[b])
+        p0, p1 = int(case.kv_page_indptr[b]), int(case.kv_page_indptr[b + 1])
+        for i in range(qlen):
+            t = q0 + i
+            ref = oracle.paged_cross_attention(case.q[t:t + 1], kp, vp, [0, 1], [0, p1 - p0],
+                                               case.kv_page_indices[p0:p1], [kvl - qlen + i + 1])
+            assert np.allclose(out[t], ref[0], atol=1e-13, rtol=0)
+
+
+def test_paged_causal_single_query_steps_are_cross_attention():
+    case, kp, vp = _causal_case(45, [1, 1, 1], [7, 16, 50])
+    causal = _causal(case, kp, vp)
+    cross = oracle.paged_cross_attention(case.q, kp, vp, case.qo_indptr, case.kv_page_indptr,
+                                         case.kv_page_indices, case.kv_len)
+    assert np.allclose(causal, cross, atol=1e-13, rtol=0)
+
+
+def test_paged_causal_rows_match_full():
+    case, kp, vp = _causal_case(47, [4, 2, 6], [30, 2, 70], hq=6, hkv=3, d=32)
+    full = _causal(case, kp, vp)
+    rows = [(0, 0), (3, 5), (4, 2), (5, 1), (11, 4)]
+    got = oracle.paged_causal_attention_rows(case.q, kp, vp, case.qo_indptr, case.kv_page_indptr,
+                                             case.kv_page_indices, case.kv_len, rows)
+    for n, (t, h) in enumerate(rows):
+        assert np.allclose(got[n], full[t, h], atol=1e-13, rtol=0)
+
+
+def _split_stream(case, n_new):
+    """The first kv_len - n tokens of every request (packed) and the last n (packed)."""
+    pre, new, cu_pre, cu_new = [], [], [0], [0]
+    for b in range(case.batch):
+        c0, c1 = int(case.cu_enc[b]), int(case.cu_enc[b + 1])
+        pre.append(torch.arange(c0, c1 - n_new[b]))
+        new.append(torch.arange(c1 - n_new[b], c1))
+        cu_pre.append(cu_pre[-1] + c1 - n_new[b] - c0)
+        cu_new.append(cu_new[-1] + n_new[b])
+    return torch.cat(pre), torch.cat(new), np.array(cu_pre), np.array(cu_new)
+
+
+def test_append_completes_the_context_write_bit_for_bit():
+    """Context write of each stream's first tokens, then the append of its last ones, leaves
+    exactly the pools of one context write of the whole streams (NaN sentinel elsewhere)."""
+    case = inputs.paged_case(46, q_lens=[3, 1, 5, 0], ctx_lens=[20, 1, 37, 16], num_qo_heads=2,
+                             num_kv_heads=2, head_dim=8, page_size=16, pool_pages=12)
+    full_k, full_v = _oracle_pools(case)
+    n_new = [3, 1, 5, 0]
+    pre, new, cu_pre, cu_new = _split_stream(case, n_new)
+    kp = inputs.nan_pool(case.num_pages, 2, 16, 8)
+    vp = inputs.nan_pool(case.num_pages, 2, 16, 8)
+    kp, vp = oracle.context_write(case.k_ctx[pre], case.v_ctx[pre], cu_pre, case.kv_page_indptr,
+                                  case.kv_page_indices, kp, vp)
+    kp, vp = oracle.append_kv(case.k_ctx[new], case.v_ctx[new], cu_new, case.kv_page_indptr,
+                              case.kv_page_indices, case.kv_len, kp, vp)
+    assert torch.equal(kp.view(torch.int16), full_k.view(torch.int16))
+    assert torch.equal(vp.view(torch.int16), full_v.view(torch.int16))
+
+
+def test_two_appends_equal_one():
+    case = inputs.paged_case(48, q_lens=[1, 1], ctx_lens=[19, 34], num_qo_heads=2,
+                             num_kv_heads=1, head_dim=8, page_size=16, pool_pages=6)
+    pre, new, cu_pre, cu_new = _split_stream(case, [3, 2])
+    kp = inputs.nan_pool(case.num_pages, 1, 16, 8)
+    vp = inputs.nan_pool(case.num_pages, 1, 16, 8)
+    kp, vp = oracle.context_write(case.k_ctx[pre], case.v_ctx[pre], cu_pre, case.kv_page_indptr,
+                                  case.kv_page_indices, kp, vp)
+    once = oracle.append_kv(case.k_ctx[new], case.v_ctx[new], cu_new, case.kv_page_indptr,
+                            case.kv_page_indices, case.kv_len, kp, vp)
+    # the same tokens in two steps: the first two of each request, then the rest
+    kl_mid = case.kv_len - np.array([1, 1])
+    first = torch.cat([new[0:2], new[3:4]])
+    second = torch.cat([new[2:3], new[4:5]])
+    kp2, vp2 = oracle.append_kv(case.k_ctx[first], case.v_ctx[first], [0, 2, 3],
+                                case.kv_page_indptr, case.kv_page_indices, kl_mid, kp, vp)
+    kp2, vp2 = oracle.append_kv(case.k_ctx[second], case.v_ctx[second], [0, 1, 2],
+                                case.kv_page_indptr, case.kv_page_indices, case.kv_len, kp2, vp2)
+    assert torch.equal(kp2.view(torch.int16), once[0].view(torch.int16))
+    assert torch.equal(vp2.view(torch.int16), once[1].view(torch.int16))
