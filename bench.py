@@ -54,7 +54,7 @@ def parse():
     ap.add_argument("--skip-workloads", action="store_true",
                     help="only the headline workload (no per-workload table)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--profile-case", type=int, default=None, choices=[1, 2, 3, 4, 5],
+    ap.add_argument("--profile-case", type=int, default=None, choices=[1, 2, 3, 4, 5, 6],
                     help="run only this workload's layer call --reps times (for ncu captures)")
     ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
@@ -80,12 +80,16 @@ def job_gbs(bytes_per_rank_step: float, world: int, ms_per_step: float) -> float
     return bytes_per_rank_step * world / (ms_per_step * 1e-3) / 1e9
 
 
-def paged_work(case):
+def paged_work(case, causal=False):
     """(flops, bytes) of one layer call: 4*d*Hq per visible (query, key) pair; valid K/V read
-    once per KV head, plus Q and O."""
+    once per KV head, plus Q and O.  Causal: query i of a request sees kv_len - qlen + i + 1
+    keys."""
     q_len = np.diff(case.qo_indptr).astype(np.int64)
     kv = case.kv_len.astype(np.int64)
-    pairs = int((q_len * kv).sum())
+    if causal:
+        pairs = int((q_len * (kv - q_len) + q_len * (q_len + 1) // 2).sum())
+    else:
+        pairs = int((q_len * kv).sum())
     flops = 4 * case.head_dim * case.num_qo_heads * pairs
     kv_tokens = int(kv[q_len > 0].sum())
     kv_bytes = kv_tokens * case.num_kv_heads * case.head_dim * 2 * 2
@@ -229,7 +233,8 @@ def setup_workload(i, dev):
     bytes, host plan µs).  Paged workloads get their context through the context write."""
     import torch
     from ragged_attention_encoder_b200 import Context, inputs
-    case = inputs.workload(i)
+    causal = i == 6
+    case = inputs.causal_chunked_prefill() if causal else inputs.workload(i)
     if hasattr(case, "kv_page_indices"):
         ctx = Context(case.num_qo_heads, case.num_kv_heads, case.head_dim, case.page_size,
                       device=dev)
@@ -240,12 +245,12 @@ def setup_workload(i, dev):
         torch.cuda.synchronize()
         t0 = time.perf_counter()
         plan = ctx.plan_paged(case.qo_indptr, case.kv_page_indptr, case.kv_page_indices,
-                              case.kv_len, case.num_pages)
+                              case.kv_len, case.num_pages, causal=causal)
         plan_us = (time.perf_counter() - t0) * 1e6
         q = case.q.to(dev)
         out = torch.empty_like(q)
         call = lambda: ctx.run_paged(plan, q, kp, vp, out)  # noqa: E731
-        flops, nbytes, _ = paged_work(case)
+        flops, nbytes, _ = paged_work(case, causal)
     else:
         ctx = Context(case.num_qo_heads, case.num_kv_heads, case.head_dim, 16, device=dev)
         torch.cuda.synchronize()
@@ -260,11 +265,12 @@ def setup_workload(i, dev):
 
 
 def workload_table(dev, peaks, flush_buf):
-    """Per-layer-call numbers of the five workloads: median of 100 calls after 10 warm-up
-    calls, L2 flushed (a 256 MB write, over twice the L2) before every call."""
+    """Per-layer-call numbers of the five workloads, and of paged causal chunked prefill (6):
+    median of 100 calls after 10 warm-up calls, L2 flushed (a 256 MB write, over twice the
+    L2) before every call."""
     import torch
     rows = {}
-    for i in (1, 2, 3, 4, 5):
+    for i in (1, 2, 3, 4, 5, 6):
         case, ctx, plan, call, flops, nbytes, plan_us = setup_workload(i, dev)
         tot, attn, merge = time_layer_calls(ctx, call, 10, 100, flush_buf)
         ctx.check_device_status()

@@ -159,6 +159,21 @@ int rae_write_context_noalloc(const void* k_src, const void* v_src, const int32_
                               void* stream);
 
 /*
+ * Append (page "mstar.engine.resources.attn.config", AttentionStep: a step's own tokens join
+ * its KV stream; page "mstar.engine.resources.attn.cross": a stream is written through
+ * ordinary Segments).  Writes the append_indptr[b+1] - append_indptr[b] new tokens of
+ * request b -- rows append_indptr[b]... of k_new, v_new [append_indptr[B], Hkv, d] (device,
+ * bf16) -- to sequence positions kv_len[b] - n_b ... kv_len[b] - 1 of its pages, where kv_len
+ * counts the request's tokens after the append.  Host int32 arrays as for rae_plan_paged;
+ * the pages must cover kv_len tokens, a page may be written by one request only per call,
+ * and nothing outside those slots is touched.  Asynchronous on `stream`; bit-exact copy.
+ */
+int rae_append_kv(rae_ctx* ctx, const void* k_new, const void* v_new,
+                  const int32_t* append_indptr, const int32_t* kv_page_indptr,
+                  const int32_t* kv_page_indices, const int32_t* kv_len, int32_t batch,
+                  void* k_pool, void* v_pool, int32_t num_pages, void* workspace, void* stream);
+
+/*
  * Plan of paged cross-attention (FlashInferCrossManager.plan; QueryPacking.qo_indptr).
  * Host int32 arrays: qo_indptr [B+1] (cumulative query lengths, qo_indptr[0] == 0),
  * kv_page_indptr [B+1], kv_page_indices [kv_page_indptr[B]], kv_len [B] (context tokens of
@@ -179,6 +194,18 @@ int rae_plan_paged(rae_ctx* ctx, int32_t slot, const int32_t* qo_indptr,
  * span).  block_size > 0: block-causal, local position i sees j iff j / bs <= i / bs (blocks
  * counted from each span's start); block_size == 0: every key of the span is visible.
  */
+/*
+ * Plan of paged causal self-attention (page "mstar.engine.resources.attn.config",
+ * AttentionStep with causal=True): the same arrays as rae_plan_paged, where the
+ * qo_indptr[b+1] - qo_indptr[b] queries of request b are the last tokens of its kv_len[b]
+ * tokens (already appended), and query i of the request sees keys 0 ... kv_len[b] - qlen + i.
+ * qlen <= kv_len for every request (RAE_ERR_INVALID_ARG otherwise).  Run with rae_run_paged.
+ */
+int rae_plan_paged_causal(rae_ctx* ctx, int32_t slot, const int32_t* qo_indptr,
+                          const int32_t* kv_page_indptr, const int32_t* kv_page_indices,
+                          const int32_t* kv_len, int32_t batch, int32_t num_pages,
+                          void* workspace, void* stream, rae_plan* out);
+
 int rae_plan_ragged(rae_ctx* ctx, int32_t slot, const int32_t* cu_q, const int32_t* cu_kv,
                     int32_t num_spans, int32_t block_size, void* workspace, void* stream,
                     rae_plan* out);
@@ -235,6 +262,12 @@ int rae_plan_paged_host(const rae_config* cfg, const int32_t* qo_indptr,
                         const int32_t* kv_page_indptr, const int32_t* kv_page_indices,
                         const int32_t* kv_len, int32_t batch, int32_t num_pages, void* image,
                         size_t image_bytes, rae_plan* out, char* err, size_t err_len);
+
+int rae_plan_paged_causal_host(const rae_config* cfg, const int32_t* qo_indptr,
+                               const int32_t* kv_page_indptr, const int32_t* kv_page_indices,
+                               const int32_t* kv_len, int32_t batch, int32_t num_pages,
+                               void* image, size_t image_bytes, rae_plan* out, char* err,
+                               size_t err_len);
 
 int rae_plan_ragged_host(const rae_config* cfg, const int32_t* cu_q, const int32_t* cu_kv,
                          int32_t num_spans, int32_t block_size, void* image, size_t image_bytes,

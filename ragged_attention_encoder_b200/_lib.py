@@ -82,6 +82,9 @@ SIGNATURES = {
                                       ctypes.POINTER(RaePlan)]),
     "rae_plan_ragged": (ctypes.c_int, [vp, i32, P32, P32, i32, i32, vp, vp,
                                        ctypes.POINTER(RaePlan)]),
+    "rae_plan_paged_causal": (ctypes.c_int, [vp, i32, P32, P32, P32, P32, i32, i32, vp, vp,
+                                             ctypes.POINTER(RaePlan)]),
+    "rae_append_kv": (ctypes.c_int, [vp, vp, vp, P32, P32, P32, P32, i32, vp, vp, i32, vp, vp]),
     "rae_run_paged": (ctypes.c_int, [vp, ctypes.POINTER(RaePlan), vp, vp, vp, i32, vp,
                                      ctypes.c_float, vp, vp]),
     "rae_run_ragged": (ctypes.c_int, [vp, ctypes.POINTER(RaePlan), vp, vp, vp, i32, vp,
@@ -93,6 +96,9 @@ SIGNATURES = {
                                            ctypes.c_char_p, sz]),
     "rae_plan_ragged_host": (ctypes.c_int, [ctypes.POINTER(RaeConfig), P32, P32, i32, i32, vp,
                                             sz, ctypes.POINTER(RaePlan), ctypes.c_char_p, sz]),
+    "rae_plan_paged_causal_host": (ctypes.c_int, [ctypes.POINTER(RaeConfig), P32, P32, P32, P32,
+                                                  i32, i32, vp, sz, ctypes.POINTER(RaePlan),
+                                                  ctypes.c_char_p, sz]),
     "rae_plan_image_bytes_for": (sz, [ctypes.POINTER(RaeConfig)]),
     "rae_write_context_noalloc": (ctypes.c_int, [vp, vp, P32, P32, P32, i32, vp, vp, i32, i32,
                                                  i32, i32, vp]),

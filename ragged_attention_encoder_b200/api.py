@@ -187,8 +187,28 @@ class Context:
             _dev(v_pool, "v_pool"), int(k_pool.shape[0]), self.workspace.data_ptr(),
             _stream_handle(self.device)))
 
+    def append_kv(self, k_new, v_new, append_indptr, kv_page_indptr, kv_page_indices, kv_len,
+                  k_pool, v_pool):
+        """Writes each request's new tokens (rows append_indptr[b]... of k_new / v_new) to the
+        last positions of its kv_len[b]-token sequence (kv_len counts the appended tokens)."""
+        ap = _i32(append_indptr)
+        ip = _i32(kv_page_indptr)
+        ix = _i32(kv_page_indices)
+        kl = _i32(kv_len)
+        batch = int(kl.shape[0])
+        if ap.shape[0] != batch + 1 or ip.shape[0] != batch + 1:
+            raise ValueError("append_indptr and kv_page_indptr must have batch + 1 entries")
+        self._check(self._lib.rae_append_kv(
+            self._h, _dev(k_new, "k_new"), _dev(v_new, "v_new"), _ptr32(ap), _ptr32(ip),
+            _ptr32(ix) if ix.size else None, _ptr32(kl) if kl.size else None, batch,
+            _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"), int(k_pool.shape[0]),
+            self.workspace.data_ptr(), _stream_handle(self.device)))
+
     def plan_paged(self, qo_indptr, kv_page_indptr, kv_page_indices, kv_len, num_pages: int,
-                   slot=None) -> Plan:
+                   slot=None, causal: bool = False) -> Plan:
+        """Plan of paged attention.  causal=False: cross-attention, every query sees all
+        kv_len keys.  causal=True: the queries are the last tokens of each kv_len-token
+        sequence and query i sees keys up to its own position, kv_len - qlen + i."""
         qo = _i32(qo_indptr)
         ip = _i32(kv_page_indptr)
         ix = _i32(kv_page_indices)
@@ -197,7 +217,8 @@ class Context:
         if qo.shape[0] != batch + 1 or ip.shape[0] != batch + 1:
             raise ValueError("qo_indptr and kv_page_indptr must have batch + 1 entries")
         raw = _lib.RaePlan()
-        self._check(self._lib.rae_plan_paged(
+        fn = self._lib.rae_plan_paged_causal if causal else self._lib.rae_plan_paged
+        self._check(fn(
             self._h, self._slot(slot), _ptr32(qo), _ptr32(ip), _ptr32(ix) if ix.size else None,
             _ptr32(kl) if kl.size else None, batch, int(num_pages), self.workspace.data_ptr(),
             _stream_handle(self.device), ctypes.byref(raw)))
@@ -292,7 +313,8 @@ def _decode_image(img: np.ndarray, raw: _lib.RaePlan) -> dict:
 
 
 def plan_paged_host(qo_indptr, kv_page_indptr, kv_page_indices, kv_len, num_pages, *,
-                    num_qo_heads, num_kv_heads, head_dim, page_size, num_sms=148, **cap) -> dict:
+                    num_qo_heads, num_kv_heads, head_dim, page_size, num_sms=148, causal=False,
+                    **cap) -> dict:
     """Runs the library's host plan builder without CUDA and decodes the plan image."""
     lib = _lib.load()
     cfg = _host_cfg(num_qo_heads, num_kv_heads, head_dim, page_size, num_sms, **cap)
@@ -303,7 +325,8 @@ def plan_paged_host(qo_indptr, kv_page_indptr, kv_page_indices, kv_len, num_page
     qo, ip, ix, kl = _i32(qo_indptr), _i32(kv_page_indptr), _i32(kv_page_indices), _i32(kv_len)
     raw = _lib.RaePlan()
     err = ctypes.create_string_buffer(512)
-    st = lib.rae_plan_paged_host(ctypes.byref(cfg), _ptr32(qo), _ptr32(ip),
+    fn = lib.rae_plan_paged_causal_host if causal else lib.rae_plan_paged_host
+    st = fn(ctypes.byref(cfg), _ptr32(qo), _ptr32(ip),
                                  _ptr32(ix) if ix.size else None, _ptr32(kl) if kl.size else None,
                                  int(kl.shape[0]), int(num_pages), img.ctypes.data, nbytes,
                                  ctypes.byref(raw), err, 512)

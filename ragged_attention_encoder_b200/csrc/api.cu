@@ -287,12 +287,18 @@ int rae_set_wait_timeout_ns(rae_ctx* ctx, int64_t timeout_ns) {
   return RAE_OK;
 }
 
-int rae_write_context(rae_ctx* ctx, const void* k_src, const void* v_src, const int32_t* cu_enc,
-                      const int32_t* page_indptr, const int32_t* page_indices, int32_t batch,
-                      void* k_pool, void* v_pool, int32_t num_pages, void* workspace,
-                      void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The context write and the append: the tokens of request b (rows cu_src[b]..cu_src[b+1]-1
+// of k_src / v_src) go to sequence positions start[b]... of its pages (start == nullptr: 0).
+int write_kv(rae_ctx* ctx, const void* k_src, const void* v_src, const int32_t* cu_src,
+             const int32_t* page_indptr, const int32_t* page_indices, const int32_t* start,
+             int32_t batch, void* k_pool, void* v_pool, int32_t num_pages, void* workspace,
+             void* stream) {
   if (!ctx) return RAE_ERR_INVALID_ARG;
-  if (!workspace || !k_pool || !v_pool || ((!k_src || !v_src) && batch > 0 && cu_enc && cu_enc[batch] > 0))
+  if (!workspace || !k_pool || !v_pool || ((!k_src || !v_src) && batch > 0 && cu_src && cu_src[batch] > 0))
     return set_err(ctx, RAE_ERR_INVALID_ARG, "NULL device pointer");
   if (!aligned16(k_src) || !aligned16(v_src) || !aligned16(k_pool) || !aligned16(v_pool))
     return set_err(ctx, RAE_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
@@ -300,7 +306,7 @@ int rae_write_context(rae_ctx* ctx, const void* k_src, const void* v_src, const 
   if (rc) return rc;
   std::string msg;
   int64_t n = 0;
-  rc = build_write_items(ctx->cfg, cu_enc, page_indptr, page_indices, batch, num_pages,
+  rc = build_write_items(ctx->cfg, cu_src, page_indptr, page_indices, start, batch, num_pages,
                          ctx->host_write, ctx->cfg.max_kv_pages, &n, &msg);
   if (rc) return set_err(ctx, rc, msg);
   if (n == 0) return RAE_OK;
@@ -317,6 +323,40 @@ int rae_write_context(rae_ctx* ctx, const void* k_src, const void* v_src, const 
   return RAE_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+int rae_write_context(rae_ctx* ctx, const void* k_src, const void* v_src, const int32_t* cu_enc,
+                      const int32_t* page_indptr, const int32_t* page_indices, int32_t batch,
+                      void* k_pool, void* v_pool, int32_t num_pages, void* workspace,
+                      void* stream) {
+  return write_kv(ctx, k_src, v_src, cu_enc, page_indptr, page_indices, nullptr, batch, k_pool,
+                  v_pool, num_pages, workspace, stream);
+}
+
+int rae_append_kv(rae_ctx* ctx, const void* k_new, const void* v_new,
+                  const int32_t* append_indptr, const int32_t* kv_page_indptr,
+                  const int32_t* kv_page_indices, const int32_t* kv_len, int32_t batch,
+                  void* k_pool, void* v_pool, int32_t num_pages, void* workspace, void* stream) {
+  if (!ctx) return RAE_ERR_INVALID_ARG;
+  if (batch < 0) return set_err(ctx, RAE_ERR_INVALID_ARG, "batch < 0");
+  if (batch > ctx->cfg.max_batch) return set_err(ctx, RAE_ERR_CAPACITY, "batch > max_batch");
+  if (batch > 0 && (!append_indptr || !kv_len))
+    return set_err(ctx, RAE_ERR_INVALID_ARG, "append_indptr or kv_len is NULL");
+  std::vector<int32_t> start(size_t(batch > 0 ? batch : 0));
+  for (int32_t b = 0; b < batch; ++b) {
+    const int32_t n = append_indptr[b + 1] - append_indptr[b];
+    if (n < 0) return set_err(ctx, RAE_ERR_INVALID_ARG, "append_indptr decreases");
+    if (n > kv_len[b])
+      return set_err(ctx, RAE_ERR_INVALID_ARG,
+                     "request " + std::to_string(b) + " appends more tokens than kv_len holds");
+    start[size_t(b)] = kv_len[b] - n;
+  }
+  return write_kv(ctx, k_new, v_new, append_indptr, kv_page_indptr, kv_page_indices,
+                  start.data(), batch, k_pool, v_pool, num_pages, workspace, stream);
+}
+
 int rae_plan_paged(rae_ctx* ctx, int32_t slot, const int32_t* qo_indptr,
                    const int32_t* kv_page_indptr, const int32_t* kv_page_indices,
                    const int32_t* kv_len, int32_t batch, int32_t num_pages, void* workspace,
@@ -330,6 +370,26 @@ int rae_plan_paged(rae_ctx* ctx, int32_t slot, const int32_t* qo_indptr,
   rae_plan plan{};
   rc = build_paged_plan(ctx->cfg, qo_indptr, kv_page_indptr, kv_page_indices, kv_len, batch,
                         num_pages, ctx->host_slot[slot], ctx->image_words, &plan, &msg);
+  if (rc) return set_err(ctx, rc, msg);
+  rc = stage_plan(ctx, slot, workspace, stream, &plan, rc);
+  if (rc) return rc;
+  *out = plan;
+  return RAE_OK;
+}
+
+int rae_plan_paged_causal(rae_ctx* ctx, int32_t slot, const int32_t* qo_indptr,
+                          const int32_t* kv_page_indptr, const int32_t* kv_page_indices,
+                          const int32_t* kv_len, int32_t batch, int32_t num_pages,
+                          void* workspace, void* stream, rae_plan* out) {
+  if (!ctx) return RAE_ERR_INVALID_ARG;
+  if (slot != 0 && slot != 1) return set_err(ctx, RAE_ERR_INVALID_ARG, "slot must be 0 or 1");
+  if (!workspace || !out) return set_err(ctx, RAE_ERR_INVALID_ARG, "NULL workspace or out");
+  int rc = wait_staging(ctx, ctx->slot_event[slot], &ctx->slot_pending[slot]);
+  if (rc) return rc;
+  std::string msg;
+  rae_plan plan{};
+  rc = build_paged_plan(ctx->cfg, qo_indptr, kv_page_indptr, kv_page_indices, kv_len, batch,
+                        num_pages, ctx->host_slot[slot], ctx->image_words, &plan, &msg, true);
   if (rc) return set_err(ctx, rc, msg);
   rc = stage_plan(ctx, slot, workspace, stream, &plan, rc);
   if (rc) return rc;
@@ -508,6 +568,25 @@ int rae_plan_paged_host(const rae_config* cfg, const int32_t* qo_indptr,
   int rc = build_paged_plan(*cfg, qo_indptr, kv_page_indptr, kv_page_indices, kv_len, batch,
                             num_pages, static_cast<int32_t*>(image), int64_t(image_bytes / 4),
                             &plan, &msg);
+  if (rc) {
+    if (err && err_len) std::snprintf(err, err_len, "%s", msg.c_str());
+    return rc;
+  }
+  *out = plan;
+  return RAE_OK;
+}
+
+int rae_plan_paged_causal_host(const rae_config* cfg, const int32_t* qo_indptr,
+                               const int32_t* kv_page_indptr, const int32_t* kv_page_indices,
+                               const int32_t* kv_len, int32_t batch, int32_t num_pages,
+                               void* image, size_t image_bytes, rae_plan* out, char* err,
+                               size_t err_len) {
+  if (!cfg || !out) return RAE_ERR_INVALID_ARG;
+  std::string msg;
+  rae_plan plan{};
+  int rc = build_paged_plan(*cfg, qo_indptr, kv_page_indptr, kv_page_indices, kv_len, batch,
+                            num_pages, static_cast<int32_t*>(image), int64_t(image_bytes / 4),
+                            &plan, &msg, true);
   if (rc) {
     if (err && err_len) std::snprintf(err, err_len, "%s", msg.c_str());
     return rc;

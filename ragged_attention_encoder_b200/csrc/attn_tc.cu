@@ -396,7 +396,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       const bool live = __any_sync(0xffffffffu, row_ok);
       // Keys visible to this row, as a limit on the logical key index.
       int lim = tile.kv1;
-      if (!p.paged) {
+      if (p.paged && plan.block_size > 0) {
+        // causal plan: this query is token kv_len - qlen + i of its sequence
+        const int qlen = plan.a[tile.req + 1] - plan.a[tile.req];
+        lim = min(lim, plan.b[tile.req] - qlen + (q_tok - plan.a[tile.req]) + 1);
+      } else if (!p.paged) {
         const int lk = plan.b[tile.req + 1] - plan.b[tile.req];
         int rl = lk;
         if (plan.block_size > 0) {

@@ -48,7 +48,7 @@ __global__ void __launch_bounds__(256) context_write_kernel(const WriteItem* __r
         const int32_t rem = e - slot * per_tok;
         const int32_t h = rem / vec_per_row;
         const int32_t u = rem - h * vec_per_row;
-        const int64_t dst = page0 + (int64_t(h) * page_size + slot) * vec_per_row + u;
+        const int64_t dst = page0 + (int64_t(h) * page_size + it.slot0 + slot) * vec_per_row + u;
         __stcs(k_pool + dst, kv[i]);
         __stcs(v_pool + dst, vv[i]);
       }
@@ -135,7 +135,7 @@ extern "C" int rae_write_context_noalloc(const void* k_src, const void* v_src,
   std::string msg;
   // Sizes beyond kNoAllocMaxPages page copies come back as RAE_ERR_CAPACITY, before any
   // device work.
-  int rc = build_write_items(cfg, cu_enc, page_indptr, page_indices, batch, num_pages,
+  int rc = build_write_items(cfg, cu_enc, page_indptr, page_indices, nullptr, batch, num_pages,
                              g_noalloc_host, kNoAllocMaxPages, &n, &msg);
   if (rc) return rc;
   if (n == 0) return RAE_OK;

@@ -166,6 +166,19 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
         for (int e = 0; e < 8; ++e) qf[r][e] = 0.f;
       }
     }
+    // Keys visible to each row: the tile's range, and under a causal plan (block_size 1) the
+    // row's own position in its sequence (queries are the sequence's last tokens).
+    int lim[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      lim[r] = tile.kv1;
+      if (plan.block_size > 0 && r < rows) {
+        const int q_first = plan.a[tile.req];
+        const int qlen = plan.a[tile.req + 1] - q_first;
+        const int tok = tile.q0 + r / geo.g;
+        lim[r] = min(lim[r], plan.b[tile.req] - qlen + (tok - q_first) + 1);
+      }
+    }
     float m[R], l[R], acc[R][8];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -195,7 +208,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
             kf[2 * e] = bf16lo_to_f32(w[e]);
             kf[2 * e + 1] = bf16hi_to_f32(w[e]);
           }
-          const bool valid = kbase + i * C::KPI + grp < tile.kv1;
+          const int key = kbase + i * C::KPI + grp;
 #pragma unroll
           for (int r = 0; r < R; ++r) {
             float dot = 0.f;
@@ -203,7 +216,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
             for (int e = 0; e < 8; ++e) dot = fmaf(qf[r][e], kf[e], dot);
 #pragma unroll
             for (int o = C::CPL / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-            x[r][i] = valid ? dot * scale_log2 : -INFINITY;
+            x[r][i] = key < lim[r] ? dot * scale_log2 : -INFINITY;
           }
         }
 #pragma unroll

@@ -334,7 +334,7 @@ int64_t image_words_for(const rae_config& cfg) { return image_bound(cfg); }
 int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
                      const int32_t* kv_page_indptr, const int32_t* kv_page_indices,
                      const int32_t* kv_len, int32_t batch, int32_t num_pages, int32_t* image,
-                     int64_t image_words, rae_plan* out, std::string* err) {
+                     int64_t image_words, rae_plan* out, std::string* err, bool causal) {
   int rc = check_config(cfg, err);
   if (rc) return rc;
   if (!image) return fail(err, RAE_ERR_INVALID_ARG, "image is NULL");
@@ -363,6 +363,9 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
     if (kv_page_indptr[b + 1] - kv_page_indptr[b] < need)
       return fail(err, RAE_ERR_INVALID_ARG,
                   "request " + std::to_string(b) + " has fewer pages than kv_len needs");
+    if (causal && qo_indptr[b + 1] - qo_indptr[b] > kv_len[b])
+      return fail(err, RAE_ERR_INVALID_ARG,
+                  "request " + std::to_string(b) + " has more queries than sequence tokens");
   }
 
   const int32_t g = cfg.num_qo_heads / cfg.num_kv_heads;
@@ -373,7 +376,8 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
   const int64_t max_rows = int64_t(max_qlen) * g;
   const bool simt = max_rows <= kSimtMaxRows;
   const int32_t swap_n = max_rows <= 32 ? 32 : 64;
-  const bool swap = !simt && cfg.head_dim == 128 && max_rows <= 64 && swap_n % g == 0;
+  // (causal plans use the two families that apply a per-row key limit)
+  const bool swap = !causal && !simt && cfg.head_dim == 128 && max_rows <= 64 && swap_n % g == 0;
   const int32_t kind = simt ? kKindDecodeSimt : (swap ? kKindTcPagedSwap : kKindTcPaged);
   // tcgen05 units hold up to two 128-row query tiles that share every K/V block.
   const int32_t tile_tok = kTcRows / g;
@@ -390,7 +394,9 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
         u.kvh = h;
         u.q0 = qo_indptr[b] + t;
         u.qn = std::min(tok_per_unit, qlen - t);
-        u.nkeys = kv_len[b];
+        // causal: the unit's last query (local index t + qn - 1) sees kv_len - qlen + t + qn
+        // keys; no row of the unit sees more
+        u.nkeys = causal ? kv_len[b] - qlen + t + u.qn : kv_len[b];
         u.rows = u.qn * g;
         u.w = (simt || swap) ? 1 : int32_t(ceil_div(u.qn, tile_tok));
         u.group = int64_t(b) * cfg.num_kv_heads + h;
@@ -400,7 +406,7 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
 
   out->batch = batch;
   out->total_q = total_q;
-  out->block_size = 0;
+  out->block_size = causal ? 1 : 0;
   int32_t rows_max = 0;
   for (const Unit& u : units) rows_max = std::max(rows_max, u.rows);
   if (swap) rows_max = swap_n;   // the row count the swapped kernel is instantiated for
@@ -416,7 +422,7 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
   if (rc) return rc;
   image[kHdrBatch] = batch;
   image[kHdrTotalQ] = total_q;
-  image[kHdrBlockSize] = 0;
+  image[kHdrBlockSize] = causal ? 1 : 0;   // paged: 1 = causal, queries at the sequence end
   image[kHdrRowsMax] = rows_max;
   return RAE_OK;
 }
@@ -482,8 +488,9 @@ int build_ragged_plan(const rae_config& cfg, const int32_t* cu_q, const int32_t*
 }
 
 int build_write_items(const rae_config& cfg, const int32_t* cu_enc, const int32_t* page_indptr,
-                      const int32_t* page_indices, int32_t batch, int32_t num_pages,
-                      WriteItem* items, int64_t max_items, int64_t* num_items, std::string* err) {
+                      const int32_t* page_indices, const int32_t* start, int32_t batch,
+                      int32_t num_pages, WriteItem* items, int64_t max_items, int64_t* num_items,
+                      std::string* err) {
   int rc = check_config(cfg, err);
   if (rc) return rc;
   if (batch < 0) return fail(err, RAE_ERR_INVALID_ARG, "batch < 0");
@@ -497,14 +504,19 @@ int build_write_items(const rae_config& cfg, const int32_t* cu_enc, const int32_
     return fail(err, RAE_ERR_CAPACITY, "pool rows overflow int32");
   std::vector<uint8_t> used(size_t(num_pages), 0);
   int64_t n = 0;
+  const int32_t P = cfg.page_size;
   for (int32_t b = 0; b < batch; ++b) {
     const int32_t len = cu_enc[b + 1] - cu_enc[b];
-    const int64_t need = ceil_div(len, cfg.page_size);
-    if (page_indptr[b + 1] - page_indptr[b] < need)
+    const int32_t pos0 = start ? start[b] : 0;
+    if (pos0 < 0) return fail(err, RAE_ERR_INVALID_ARG, "first position < 0");
+    if (len == 0) continue;
+    const int64_t end = int64_t(pos0) + len;
+    if (page_indptr[b + 1] - page_indptr[b] < ceil_div(end, P))
       return fail(err, RAE_ERR_INVALID_ARG,
-                  "request " + std::to_string(b) + " has fewer pages than its context needs");
-    for (int64_t i = 0; i < need; ++i) {
-      const int32_t page = page_indices[page_indptr[b] + i];
+                  "request " + std::to_string(b) + " has fewer pages than its tokens need");
+    for (int64_t pos = pos0; pos < end;) {
+      const int64_t lp = pos / P;
+      const int32_t page = page_indices[page_indptr[b] + lp];
       if (page < 0 || page >= num_pages)
         return fail(err, RAE_ERR_INVALID_ARG, "page id " + std::to_string(page) + " out of range");
       if (used[size_t(page)])
@@ -513,10 +525,11 @@ int build_write_items(const rae_config& cfg, const int32_t* cu_enc, const int32_
       used[size_t(page)] = 1;
       if (n >= max_items) return fail(err, RAE_ERR_CAPACITY, "write needs more pages than max_kv_pages");
       WriteItem& it = items[n++];
-      it.src_row = cu_enc[b] + int32_t(i) * cfg.page_size;
-      it.ntok = std::min<int32_t>(cfg.page_size, len - int32_t(i) * cfg.page_size);
+      it.slot0 = int32_t(pos - lp * P);
+      it.ntok = int32_t(std::min<int64_t>(P - it.slot0, end - pos));
+      it.src_row = cu_enc[b] + int32_t(pos - pos0);
       it.page = page;
-      it.pad = 0;
+      pos += it.ntok;
     }
   }
   *num_items = n;

@@ -226,6 +226,15 @@ WORKLOADS = {
 }
 
 
+def causal_chunked_prefill() -> PagedCase:
+    """Paged causal self-attention, chunked prefill: 32 requests each append a 128-token
+    chunk that closes a stream of U[256, 4096] tokens (the chunk included); 32 query heads /
+    8 KV heads, head_dim 128, pages of 16 tokens, bf16 N(0,1), random page table."""
+    return paged_case(6, q_lens=[128] * 32, ctx_lens=(256, 4096, 32), num_qo_heads=32,
+                      num_kv_heads=8, head_dim=128, page_size=16,
+                      name="paged_causal_chunked_prefill")
+
+
 def workload(i: int):
     return WORKLOADS[i]()
 

@@ -241,3 +241,70 @@ def test_empty_inputs_plan_nothing():
                         page_size=16)
     t = p["tiles"]
     assert t.shape[0] == 2 and np.all(t[:, 4] == 0) and np.all(t[:, 5] == 0)
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("hq,hkv,d,P", [(4, 2, 64, 16), (8, 1, 128, 32), (32, 8, 128, 16),
+                                        (64, 8, 128, 64)])
+def test_causal_paged_plan_covers_each_visible_pair_once(seed, hq, hkv, d, P):
+    """Query i of a request (stream token kv_len - qlen + i) needs keys [0, kv_len - qlen + i]:
+    each exactly once; keys past it may appear in its tile (the kernel masks them) but never
+    twice, and no tile reaches past the unit's last query."""
+    rng = np.random.default_rng(seed * 31 + hq)
+    B = int(rng.integers(1, 6))
+    kv_len = rng.integers(1, 700, B)
+    q_len = np.minimum(kv_len, rng.integers(0, 90 if seed % 2 else 4, B))
+    pages_per = (kv_len + P - 1) // P
+    indptr = np.concatenate([[0], np.cumsum(pages_per)]).astype(np.int32)
+    num_pages = int(indptr[-1]) + 3
+    indices = rng.permutation(num_pages)[: indptr[-1]].astype(np.int32)
+    qo = np.concatenate([[0], np.cumsum(q_len)]).astype(np.int32)
+    p = plan_paged_host(qo, indptr, indices, kv_len, num_pages, num_qo_heads=hq,
+                        num_kv_heads=hkv, head_dim=d, page_size=P,
+                        num_sms=int(rng.integers(1, 9)), causal=True)
+    assert p["raw"].kind in (1, 2) and p["header"][7] == 1
+    g = hq // hkv
+    _check_cta_ptr(p)
+    cover = {}
+    for tok, head, kv0, kv1, i in _tiles_rows(p["tiles"], g):
+        cover.setdefault((tok, head), []).append((kv0, kv1))
+    for b in range(B):
+        for tok in range(qo[b], qo[b + 1]):
+            lim = int(kv_len[b] - q_len[b] + (tok - qo[b]) + 1)
+            for head in range(hq):
+                keys = np.zeros(int(kv_len[b]), dtype=int)
+                for kv0, kv1 in cover.pop((tok, head)):
+                    assert 0 <= kv0 <= kv1 <= kv_len[b]
+                    keys[kv0:kv1] += 1
+                assert np.all(keys[:lim] == 1) and np.all(keys <= 1)
+    assert not cover
+    _check_merge(p, g, hq)
+
+
+def test_causal_plan_rejects_more_queries_than_stream_tokens():
+    with pytest.raises(ValueError, match="more queries"):
+        plan_paged_host([0, 5], [0, 1], [0], [4], 1, num_qo_heads=4, num_kv_heads=2,
+                        head_dim=64, page_size=16, causal=True)
+    # the same arrays are fine for cross-attention
+    plan_paged_host([0, 5], [0, 1], [0], [4], 1, num_qo_heads=4, num_kv_heads=2, head_dim=64,
+                    page_size=16)
+
+
+def test_causal_plan_trims_key_ranges_to_the_last_query():
+    """A 64-token chunk at the start of a 4096-token stream needs only its first 64 keys."""
+    qo = np.array([0, 64], np.int32)
+    kv_len = np.array([64], np.int32)
+    ip = np.array([0, 4], np.int32)
+    p = plan_paged_host(qo, ip, np.arange(4, dtype=np.int32), kv_len, 4, num_qo_heads=32,
+                        num_kv_heads=8, head_dim=128, page_size=16, causal=True)
+    t = p["tiles"]
+    assert p["raw"].kind == 2 and np.all(t[:, 5] <= 64)
+    # 128 new tokens closing a 1128-token stream, GQA 4: units of 64 tokens (two 32-token
+    # tiles); unit u's last query is stream token 1000 + 64 (u + 1) - 1
+    qo = np.array([0, 128], np.int32)
+    kv_len = np.array([1128], np.int32)
+    ip = np.array([0, 71], np.int32)
+    p = plan_paged_host(qo, ip, np.arange(71, dtype=np.int32), kv_len, 71, num_qo_heads=8,
+                        num_kv_heads=2, head_dim=128, page_size=16, causal=True, num_sms=1)
+    ends = sorted({(int(r[2]), int(r[5])) for r in p["tiles"]})
+    assert ends == [(0, 1064), (64, 1128)]
