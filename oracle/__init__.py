@@ -29,6 +29,7 @@ from .attention import (  # noqa: F401
     paged_cross_attention,
     paged_cross_attention_rows,
     partial_attention_with_lse,
+    project_kv,
     ragged_block_causal_attention,
     ragged_block_causal_rows,
     ragged_cross_attention,

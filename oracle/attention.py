@@ -172,6 +172,22 @@ def context_write(k_src: torch.Tensor, v_src: torch.Tensor, cu_enc, page_indptr,
     return k_out, v_out
 
 
+def project_kv(hidden, w_k, b_k, w_v, b_v, num_kv_heads: int, head_dim: int):
+    """K and V of the encoder context (mstar.model.components.attention,
+    ``CrossAttention.compute_kv``): each packed encoder row ``x`` [hidden] goes through the K
+    and V linears, ``k = x W_k^T (+ b_k)`` and ``v = x W_v^T (+ b_v)`` with nn.Linear weights
+    ``[num_kv_heads * head_dim, hidden]``; float64; returned as [tokens, Hkv, d] each."""
+    x = as_f64(hidden)
+    k = x @ as_f64(w_k).T
+    v = x @ as_f64(w_v).T
+    if b_k is not None:
+        k = k + as_f64(b_k)[None, :]
+    if b_v is not None:
+        v = v + as_f64(b_v)[None, :]
+    return (k.reshape(x.shape[0], num_kv_heads, head_dim),
+            v.reshape(x.shape[0], num_kv_heads, head_dim))
+
+
 def append_kv(k_new: torch.Tensor, v_new: torch.Tensor, append_indptr, page_indptr,
               page_indices, kv_len, k_pool: torch.Tensor, v_pool: torch.Tensor):
     """Append of a step's own K/V to its stream, done by plain element copies (bit exact).

@@ -462,3 +462,50 @@ def test_two_appends_equal_one():
                                 case.kv_page_indptr, case.kv_page_indices, case.kv_len, kp2, vp2)
     assert torch.equal(kp2.view(torch.int16), once[0].view(torch.int16))
     assert torch.equal(vp2.view(torch.int16), once[1].view(torch.int16))
+
+
+# ----------------------------------------------------------- K/V projection of the context
+
+def _proj_inputs(seed, tokens, hidden, hkv, d, bias=True):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(tokens, hidden, generator=g).to(torch.bfloat16)
+    wk = (torch.randn(hkv * d, hidden, generator=g) / hidden ** 0.5).to(torch.bfloat16)
+    wv = (torch.randn(hkv * d, hidden, generator=g) / hidden ** 0.5).to(torch.bfloat16)
+    bk = torch.randn(hkv * d, generator=g).to(torch.bfloat16) if bias else None
+    bv = torch.randn(hkv * d, generator=g).to(torch.bfloat16) if bias else None
+    return x, wk, bk, wv, bv
+
+
+def test_projection_of_a_one_hot_row_is_a_weight_column():
+    """x = e_i gives k = W_k[:, i] + b_k: fixes which index of W is contracted (W is not
+    square here, so a transposed product could not even be formed)."""
+    hidden, hkv, d = 96, 2, 16
+    _, wk, bk, wv, bv = _proj_inputs(60, 1, hidden, hkv, d)
+    x = torch.eye(hidden, dtype=torch.bfloat16)[[0, 7, 95]]
+    k, v = oracle.project_kv(x, wk, bk, wv, bv, hkv, d)
+    for n, i in enumerate([0, 7, 95]):
+        assert np.array_equal(k[n].reshape(-1), oracle.as_f64(wk)[:, i] + oracle.as_f64(bk))
+        assert np.array_equal(v[n].reshape(-1), oracle.as_f64(wv)[:, i] + oracle.as_f64(bv))
+
+
+def test_projection_with_identity_weights_returns_the_rows():
+    hkv, d = 4, 16
+    x = _proj_inputs(61, 5, hkv * d, hkv, d)[0]
+    eye = torch.eye(hkv * d, dtype=torch.bfloat16)
+    k, v = oracle.project_kv(x, eye, None, eye, None, hkv, d)
+    assert np.array_equal(k, oracle.as_f64(x).reshape(5, hkv, d))
+    assert np.array_equal(v, k)
+
+
+def test_projection_is_affine_and_zero_weights_give_the_bias():
+    hidden, hkv, d = 64, 2, 32
+    x1, wk, bk, wv, bv = _proj_inputs(62, 6, hidden, hkv, d)
+    x2 = _proj_inputs(63, 6, hidden, hkv, d)[0]
+    k1, v1 = oracle.project_kv(x1, wk, bk, wv, bv, hkv, d)
+    k2, v2 = oracle.project_kv(x2, wk, bk, wv, bv, hkv, d)
+    k3, v3 = oracle.project_kv(x1.double() * 3 + x2.double(), wk, bk, wv, bv, hkv, d)
+    b = oracle.as_f64(bk).reshape(hkv, d)
+    assert np.allclose(k3 - b, 3 * (k1 - b) + (k2 - b), atol=1e-12)
+    zero = torch.zeros_like(wk)
+    k0, v0 = oracle.project_kv(x1, zero, bk, zero, None, hkv, d)
+    assert np.array_equal(k0, np.broadcast_to(b, k0.shape)) and not np.any(v0)
