@@ -264,6 +264,69 @@ def setup_workload(i, dev):
     return case, ctx, plan, call, flops, nbytes, plan_us
 
 
+def projection_row(dev, peaks, flush_buf):
+    """The Whisper-large encode step with the K/V projections fused into the context write:
+    64 x 1500 encoder tokens, hidden 1280, 20 KV heads x 64 (k unbiased, v biased), seeded
+    random weights; CUDA events around each call (median of 30 after 5 warm-ups, L2 flushed),
+    next to the unfused sequence (two torch linears, then the context write)."""
+    import torch
+    import torch.nn.functional as F
+    from ragged_attention_encoder_b200 import Context, inputs
+    case = inputs.workload(2)
+    m, hidden, hkv, d = int(case.cu_enc[-1]), 1280, 20, 64
+    gen = torch.Generator(device=dev).manual_seed(77)
+    x = torch.randn(m, hidden, generator=gen, device=dev).to(torch.bfloat16)
+    wk = (torch.randn(hkv * d, hidden, generator=gen, device=dev) / hidden ** 0.5).to(torch.bfloat16)
+    wv = (torch.randn(hkv * d, hidden, generator=gen, device=dev) / hidden ** 0.5).to(torch.bfloat16)
+    bv = torch.randn(hkv * d, generator=gen, device=dev).to(torch.bfloat16)
+    ctx = Context(hkv, hkv, d, 16, device=dev)
+    kp = torch.empty(case.num_pages, hkv, 16, d, dtype=torch.bfloat16, device=dev)
+    vp = torch.empty_like(kp)
+
+    def fused():
+        ctx.project_write_context(x, wk, None, wv, bv, case.cu_enc, case.kv_page_indptr,
+                                  case.kv_page_indices, kp, vp)
+
+    def unfused():
+        k = F.linear(x, wk).view(m, hkv, d)
+        v = F.linear(x, wv, bv).view(m, hkv, d)
+        ctx.write_context(k, v, case.cu_enc, case.kv_page_indptr, case.kv_page_indices, kp, vp)
+
+    def timed(fn):
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(30):
+            flush_l2(flush_buf)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts) * 1e-3
+    t = timed(fused)
+    ctx.check_device_status()
+    t_unfused = timed(unfused)
+    flops = 2 * m * hidden * 2 * hkv * d
+    nbytes = m * hidden * 2 + 2 * hkv * d * hidden * 2 + 2 * m * hkv * d * 2
+    tc = flops / t / 1e12
+    return {
+        "us_per_call": round(t * 1e6, 2),
+        "tflops": round(tc, 1),
+        "hbm_gbs": round(nbytes / t / 1e9, 1),
+        "bound": "tensor",
+        "tc_frac_of_measured": round(tc / peaks["tflops"], 4),
+        "tc_frac_of_measured_sustained": round(tc / peaks["tflops_sustained"], 4),
+        "tc_frac_of_spec": round(tc / SPEC_TC_TFLOPS, 4),
+        "algorithmic_flops": flops,
+        "algorithmic_bytes": nbytes,
+        "unfused_us": round(t_unfused * 1e6, 2),
+        "unfused": "torch F.linear (cuBLAS) for K and V, then the library's context write",
+    }
+
+
 def workload_table(dev, peaks, flush_buf):
     """Per-layer-call numbers of the five workloads, and of paged causal chunked prefill (6):
     median of 100 calls after 10 warm-up calls, L2 flushed (a 256 MB write, over twice the
@@ -304,6 +367,8 @@ def workload_table(dev, peaks, flush_buf):
         }
         del ctx
         torch.cuda.empty_cache()
+    rows["whisper_encode_kv_projection_write"] = projection_row(dev, peaks, flush_buf)
+    torch.cuda.empty_cache()
     return rows
 
 

@@ -159,6 +159,26 @@ int rae_write_context_noalloc(const void* k_src, const void* v_src, const int32_
                               void* stream);
 
 /*
+ * Fused K/V projection and context write (page "mstar.model.components.attention",
+ * CrossAttention.compute_kv: (enc_len, hidden) -> (k, v), each (enc_len, heads, head_dim),
+ * through nn.Linear weights; page "mstar.engine.resources.attn.cross": the context written
+ * once).  For every packed encoder token row x of `hidden` [cu_enc[B], hidden_dim] (device,
+ * bf16, row-major): k = x . w_k^T (+ b_k), v = x . w_v^T (+ b_v), with w_k, w_v
+ * [num_kv_heads * head_dim, hidden_dim] (device, bf16, nn.Linear layout) and b_k, b_v
+ * [num_kv_heads * head_dim] bf16 or NULL; fp32 accumulation, one bf16 rounding.  Token t of
+ * request b is stored where rae_write_context would store row cu_enc[b] + t (same host arrays
+ * and checks), so the projected K/V are never materialised elsewhere.  Requires
+ * hidden_dim % 64 == 0 and num_kv_heads * head_dim % 128 == 0 (RAE_ERR_UNSUPPORTED
+ * otherwise); every device buffer 16-byte aligned; at most 8388480 tokens.  Asynchronous on
+ * `stream`.
+ */
+int rae_project_write_context(rae_ctx* ctx, const void* hidden, int32_t hidden_dim,
+                              const void* w_k, const void* b_k, const void* w_v, const void* b_v,
+                              const int32_t* cu_enc, const int32_t* page_indptr,
+                              const int32_t* page_indices, int32_t batch, void* k_pool,
+                              void* v_pool, int32_t num_pages, void* workspace, void* stream);
+
+/*
  * Append (page "mstar.engine.resources.attn.config", AttentionStep: a step's own tokens join
  * its KV stream; page "mstar.engine.resources.attn.cross": a stream is written through
  * ordinary Segments).  Writes the append_indptr[b+1] - append_indptr[b] new tokens of

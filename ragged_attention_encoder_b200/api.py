@@ -187,6 +187,33 @@ class Context:
             _dev(v_pool, "v_pool"), int(k_pool.shape[0]), self.workspace.data_ptr(),
             _stream_handle(self.device)))
 
+    def project_write_context(self, hidden, w_k, b_k, w_v, b_v, cu_enc, page_indptr,
+                              page_indices, k_pool, v_pool):
+        """Encode step with the K/V projections fused in: k = hidden . w_k^T (+ b_k) and
+        v = hidden . w_v^T (+ b_v) for every packed token, stored straight into the pages.
+        hidden [sum_enc, H]; w_k, w_v [Hkv * d, H] (nn.Linear layout); biases [Hkv * d] or
+        None; all bf16 on the device."""
+        cu = _i32(cu_enc)
+        ip = _i32(page_indptr)
+        ix = _i32(page_indices)
+        batch = int(cu.shape[0] - 1)
+        if ip.shape[0] != batch + 1:
+            raise ValueError("page_indptr must have batch + 1 entries")
+        n_out = self.num_kv_heads * self.head_dim
+        if hidden.dim() != 2 or w_k.shape != (n_out, hidden.shape[1]) or w_v.shape != w_k.shape:
+            raise ValueError("hidden must be [tokens, H] and w_k, w_v [num_kv_heads * head_dim, H]")
+        if hidden.shape[0] != int(cu[-1]):
+            raise ValueError("hidden must have cu_enc[-1] rows")
+        for b, name in ((b_k, "b_k"), (b_v, "b_v")):
+            if b is not None and tuple(b.shape) != (n_out,):
+                raise ValueError(f"{name} must have num_kv_heads * head_dim entries")
+        self._check(self._lib.rae_project_write_context(
+            self._h, _dev(hidden, "hidden"), int(hidden.shape[1]), _dev(w_k, "w_k"),
+            None if b_k is None else _dev(b_k, "b_k"), _dev(w_v, "w_v"),
+            None if b_v is None else _dev(b_v, "b_v"), _ptr32(cu), _ptr32(ip),
+            _ptr32(ix) if ix.size else None, batch, _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
+            int(k_pool.shape[0]), self.workspace.data_ptr(), _stream_handle(self.device)))
+
     def append_kv(self, k_new, v_new, append_indptr, kv_page_indptr, kv_page_indices, kv_len,
                   k_pool, v_pool):
         """Writes each request's new tokens (rows append_indptr[b]... of k_new / v_new) to the

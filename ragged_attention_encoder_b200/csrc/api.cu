@@ -293,6 +293,31 @@ namespace {
 
 // The context write and the append: the tokens of request b (rows cu_src[b]..cu_src[b+1]-1
 // of k_src / v_src) go to sequence positions start[b]... of its pages (start == nullptr: 0).
+// Validates a K/V write, lists its page copies and stages them in the workspace on `stream`;
+// *dev_items / *num_items describe the staged list (num_items 0: nothing to write).
+int stage_write_items(rae_ctx* ctx, const int32_t* cu_src, const int32_t* page_indptr,
+                      const int32_t* page_indices, const int32_t* start, int32_t batch,
+                      int32_t num_pages, void* workspace, cudaStream_t st,
+                      WriteItem** dev_items, int64_t* num_items) {
+  int rc = wait_staging(ctx, ctx->write_event, &ctx->write_pending);
+  if (rc) return rc;
+  std::string msg;
+  int64_t n = 0;
+  rc = build_write_items(ctx->cfg, cu_src, page_indptr, page_indices, start, batch, num_pages,
+                         ctx->host_write, ctx->cfg.max_kv_pages, &n, &msg);
+  if (rc) return set_err(ctx, rc, msg);
+  *num_items = n;
+  *dev_items = reinterpret_cast<WriteItem*>(static_cast<uint8_t*>(workspace) + ctx->off_write);
+  if (n == 0) return RAE_OK;
+  cudaError_t e = cudaMemcpyAsync(*dev_items, ctx->host_write, size_t(n) * sizeof(WriteItem),
+                                  cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_err(ctx, e, "write items copy");
+  e = cudaEventRecord(ctx->write_event, st);
+  if (e != cudaSuccess) return cuda_err(ctx, e, "cudaEventRecord");
+  ctx->write_pending = true;
+  return RAE_OK;
+}
+
 int write_kv(rae_ctx* ctx, const void* k_src, const void* v_src, const int32_t* cu_src,
              const int32_t* page_indptr, const int32_t* page_indices, const int32_t* start,
              int32_t batch, void* k_pool, void* v_pool, int32_t num_pages, void* workspace,
@@ -302,23 +327,13 @@ int write_kv(rae_ctx* ctx, const void* k_src, const void* v_src, const int32_t* 
     return set_err(ctx, RAE_ERR_INVALID_ARG, "NULL device pointer");
   if (!aligned16(k_src) || !aligned16(v_src) || !aligned16(k_pool) || !aligned16(v_pool))
     return set_err(ctx, RAE_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
-  int rc = wait_staging(ctx, ctx->write_event, &ctx->write_pending);
-  if (rc) return rc;
-  std::string msg;
-  int64_t n = 0;
-  rc = build_write_items(ctx->cfg, cu_src, page_indptr, page_indices, start, batch, num_pages,
-                         ctx->host_write, ctx->cfg.max_kv_pages, &n, &msg);
-  if (rc) return set_err(ctx, rc, msg);
-  if (n == 0) return RAE_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  WriteItem* dev_items = reinterpret_cast<WriteItem*>(static_cast<uint8_t*>(workspace) + ctx->off_write);
-  cudaError_t e = cudaMemcpyAsync(dev_items, ctx->host_write, size_t(n) * sizeof(WriteItem),
-                                  cudaMemcpyHostToDevice, st);
-  if (e != cudaSuccess) return cuda_err(ctx, e, "write items copy");
-  e = cudaEventRecord(ctx->write_event, st);
-  if (e != cudaSuccess) return cuda_err(ctx, e, "cudaEventRecord");
-  ctx->write_pending = true;
-  e = launch_context_write(dev_items, n, k_src, v_src, k_pool, v_pool, geometry(ctx->cfg), st);
+  WriteItem* dev_items = nullptr;
+  int64_t n = 0;
+  int rc = stage_write_items(ctx, cu_src, page_indptr, page_indices, start, batch, num_pages,
+                             workspace, st, &dev_items, &n);
+  if (rc || n == 0) return rc;
+  cudaError_t e = launch_context_write(dev_items, n, k_src, v_src, k_pool, v_pool, geometry(ctx->cfg), st);
   if (e != cudaSuccess) return cuda_err(ctx, e, "context write launch");
   return RAE_OK;
 }
@@ -333,6 +348,61 @@ int rae_write_context(rae_ctx* ctx, const void* k_src, const void* v_src, const 
                       void* stream) {
   return write_kv(ctx, k_src, v_src, cu_enc, page_indptr, page_indices, nullptr, batch, k_pool,
                   v_pool, num_pages, workspace, stream);
+}
+
+int rae_project_write_context(rae_ctx* ctx, const void* hidden, int32_t hidden_dim,
+                              const void* w_k, const void* b_k, const void* w_v, const void* b_v,
+                              const int32_t* cu_enc, const int32_t* page_indptr,
+                              const int32_t* page_indices, int32_t batch, void* k_pool,
+                              void* v_pool, int32_t num_pages, void* workspace, void* stream) {
+  if (!ctx) return RAE_ERR_INVALID_ARG;
+  const rae_config& c = ctx->cfg;
+  const int32_t n_half = c.num_kv_heads * c.head_dim;
+  if (hidden_dim <= 0 || hidden_dim % 64 != 0 || n_half % 128 != 0)
+    return set_err(ctx, RAE_ERR_UNSUPPORTED,
+                   "projection needs hidden_dim % 64 == 0 and num_kv_heads * head_dim % 128 == 0");
+  if (!workspace || !k_pool || !v_pool || !w_k || !w_v)
+    return set_err(ctx, RAE_ERR_INVALID_ARG, "NULL device pointer");
+  if (!aligned16(hidden) || !aligned16(w_k) || !aligned16(w_v) || !aligned16(b_k) ||
+      !aligned16(b_v) || !aligned16(k_pool) || !aligned16(v_pool))
+    return set_err(ctx, RAE_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
+  if (batch < 0 || (batch > 0 && !cu_enc)) return set_err(ctx, RAE_ERR_INVALID_ARG, "bad cu_enc");
+  const int64_t m = batch > 0 ? cu_enc[batch] : 0;
+  if (m > int64_t(65535) * 128) return set_err(ctx, RAE_ERR_CAPACITY, "more than 8388480 tokens");
+  if (m > 0 && !hidden) return set_err(ctx, RAE_ERR_INVALID_ARG, "NULL hidden states");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WriteItem* dev_items = nullptr;
+  int64_t n = 0;
+  int rc = stage_write_items(ctx, cu_enc, page_indptr, page_indices, nullptr, batch, num_pages,
+                             workspace, st, &dev_items, &n);
+  if (rc || n == 0) return rc;
+  ProjectWriteArgs a;
+  {
+    const cuuint64_t dims[2] = {cuuint64_t(hidden_dim), cuuint64_t(m)};
+    const cuuint64_t strides[1] = {cuuint64_t(hidden_dim) * 2};
+    const cuuint32_t box[2] = {64, 128};
+    if ((rc = make_map(ctx, &a.maps[0], hidden, 2, dims, strides, box))) return rc;
+  }
+  for (int w = 0; w < 2; ++w) {
+    const cuuint64_t dims[2] = {cuuint64_t(hidden_dim), cuuint64_t(n_half)};
+    const cuuint64_t strides[1] = {cuuint64_t(hidden_dim) * 2};
+    const cuuint32_t box[2] = {64, cuuint32_t(project_write_tile_cols(n_half))};
+    if ((rc = make_map(ctx, &a.maps[1 + w], w ? w_v : w_k, 2, dims, strides, box))) return rc;
+  }
+  a.bias_k = b_k;
+  a.bias_v = b_v;
+  a.items = dev_items;
+  a.num_items = n;
+  a.k_pool = k_pool;
+  a.v_pool = v_pool;
+  a.err = reinterpret_cast<int*>(workspace);
+  a.timeout_ns = ctx->timeout_ns;
+  a.m = int32_t(m);
+  a.hidden = hidden_dim;
+  a.geo = geometry(c);
+  cudaError_t e = launch_project_write(a, st);
+  if (e != cudaSuccess) return cuda_err(ctx, e, "projection kernel launch");
+  return RAE_OK;
 }
 
 int rae_append_kv(rae_ctx* ctx, const void* k_new, const void* v_new,

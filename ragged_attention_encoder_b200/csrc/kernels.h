@@ -73,4 +73,24 @@ cudaError_t launch_attn_swapab(const DevPlan& plan, const Geometry& geo, int n_r
                                const TcTensors& maps, void* out, float* part_o, float* part_lse,
                                int* err, float scale_log2, int64_t timeout_ns, cudaStream_t stream);
 
+// Fused K/V projection and context write: [K | V] = hidden . [w_k | w_v]^T (+ bias) on
+// tcgen05, each token's row stored into its page slot.
+struct ProjectWriteArgs {
+  CUtensorMap maps[3];       // hidden {H, M} box {64, 128}; w_k, w_v {H, Hkv*d} box {64, tile cols}
+  const void* bias_k;        // [Hkv*d] bf16 or null
+  const void* bias_v;
+  const WriteItem* items;    // device page copies, in token order
+  int64_t num_items;
+  void* k_pool;
+  void* v_pool;
+  int* err;
+  int64_t timeout_ns;
+  int32_t m;                 // tokens
+  int32_t hidden;            // H, a multiple of 64
+  Geometry geo;
+};
+cudaError_t launch_project_write(const ProjectWriteArgs& args, cudaStream_t stream);
+// Output columns per tile of the projection kernel (the weight maps' box height).
+int project_write_tile_cols(int n_half);
+
 }  // namespace rae
