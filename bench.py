@@ -54,8 +54,9 @@ def parse():
     ap.add_argument("--skip-workloads", action="store_true",
                     help="only the headline workload (no per-workload table)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--profile-case", type=int, default=None, choices=[1, 2, 3, 4, 5, 6],
-                    help="run only this workload's layer call --reps times (for ncu captures)")
+    ap.add_argument("--profile-case", type=int, default=None, choices=[1, 2, 3, 4, 5, 6, 7],
+                    help="run only this workload's layer call --reps times (for ncu captures); "
+                         "6: paged causal chunked prefill, 7: the fused K/V projection")
     ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
 
@@ -264,13 +265,9 @@ def setup_workload(i, dev):
     return case, ctx, plan, call, flops, nbytes, plan_us
 
 
-def projection_row(dev, peaks, flush_buf):
-    """The Whisper-large encode step with the K/V projections fused into the context write:
-    64 x 1500 encoder tokens, hidden 1280, 20 KV heads x 64 (k unbiased, v biased), seeded
-    random weights; CUDA events around each call (median of 30 after 5 warm-ups, L2 flushed),
-    next to the unfused sequence (two torch linears, then the context write)."""
+def projection_setup(dev):
+    """Inputs of the Whisper-large encode step with fused K/V projection; returns the call."""
     import torch
-    import torch.nn.functional as F
     from ragged_attention_encoder_b200 import Context, inputs
     case = inputs.workload(2)
     m, hidden, hkv, d = int(case.cu_enc[-1]), 1280, 20, 64
@@ -286,6 +283,19 @@ def projection_row(dev, peaks, flush_buf):
     def fused():
         ctx.project_write_context(x, wk, None, wv, bv, case.cu_enc, case.kv_page_indptr,
                                   case.kv_page_indices, kp, vp)
+    return case, ctx, x, wk, wv, bv, kp, vp, fused
+
+
+def projection_row(dev, peaks, flush_buf):
+    """The Whisper-large encode step with the K/V projections fused into the context write:
+    64 x 1500 encoder tokens, hidden 1280, 20 KV heads x 64 (k unbiased, v biased), seeded
+    random weights; CUDA events around each call (median of 30 after 5 warm-ups, L2 flushed),
+    next to the unfused sequence (two torch linears, then the context write)."""
+    import torch
+    import torch.nn.functional as F
+    case, ctx, x, wk, wv, bv, kp, vp, fused = projection_setup(dev)
+    m, hkv, d = int(case.cu_enc[-1]), 20, 64
+    hidden = x.shape[1]
 
     def unfused():
         k = F.linear(x, wk).view(m, hkv, d)
@@ -695,13 +705,18 @@ def run_profile_case(args):
     import torch
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    case, ctx, plan, call, _, _, _ = setup_workload(args.profile_case, dev)
+    if args.profile_case == 7:
+        case, ctx, *_, call = projection_setup(dev)
+        info = {"profile_case": "whisper_encode_kv_projection_write"}
+    else:
+        case, ctx, plan, call, _, _, _ = setup_workload(args.profile_case, dev)
+        info = {"profile_case": case.name, "kind": plan.kernel_kind, "tiles": plan.num_tiles,
+                "ctas": plan.num_ctas}
     for _ in range(args.reps):
         call()
     torch.cuda.synchronize()
     ctx.check_device_status()
-    print(json.dumps({"profile_case": case.name, "reps": args.reps, "kind": plan.kernel_kind,
-                      "tiles": plan.num_tiles, "ctas": plan.num_ctas}), flush=True)
+    print(json.dumps({**info, "reps": args.reps}), flush=True)
 
 
 def main():
