@@ -308,3 +308,19 @@ def test_causal_plan_trims_key_ranges_to_the_last_query():
                         num_kv_heads=2, head_dim=128, page_size=16, causal=True, num_sms=1)
     ends = sorted({(int(r[2]), int(r[5])) for r in p["tiles"]})
     assert ends == [(0, 1064), (64, 1128)]
+
+
+def test_missing_library_fails_loudly():
+    """Without the built library the binding raises: there is no CPU fallback."""
+    import subprocess
+    import sys
+    code = ("import ragged_attention_encoder_b200._lib as L\n"
+            "L.LIB_PATH = L.LIB_PATH + '.absent'\n"
+            "L._lib = None\n"
+            "try:\n"
+            "    L.load()\n"
+            "except ImportError as e:\n"
+            "    print('raised', 'is missing' in str(e))\n")
+    res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
+                         timeout=120)
+    assert res.stdout.strip() == "raised True", res.stdout + res.stderr
