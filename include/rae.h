@@ -11,7 +11,13 @@
  *     (QueryPacking);
  *   - cacheless ragged block-causal self-attention within each span of one packed forward
  *     (page "mstar.engine.resources.attn.ragged.base", RaggedBlockCausalAttnManager);
- *   - cacheless two-span cross-attention per request (same page, RaggedCrossAttnManager).
+ *   - cacheless two-span cross-attention per request (same page, RaggedCrossAttnManager);
+ *   - paged causal self-attention of a step's queries over their own KV stream, after the
+ *     step's K/V are appended to it (page "mstar.engine.resources.attn.config",
+ *     AttentionStep with causal=True);
+ *
+ * and writes the context K/V into the pages, plain (the encode step) or with the K/V
+ * projections fused in (page "mstar.model.components.attention", CrossAttention.compute_kv).
  *
  * GQA follows the model page ("mstar.model.components.attention", Attention: fewer KV heads
  * than query heads); query head h reads KV head h / (Hq / Hkv).
@@ -42,7 +48,9 @@
  *       k_pool, v_pool [num_pages, Hkv, page_size, head_dim]   (paged calls)
  *       k, v           [total_kv, Hkv, head_dim]              (ragged calls)
  *     All device buffers must be 16-byte aligned; torch allocations are.
- *   - One rae_ctx may be used from one host thread at a time.
+ *   - One rae_ctx may be used from one host thread at a time.  Calls given the same
+ *     workspace share its split partials, arrival counters and error word: their device work
+ *     must not overlap (one stream per context, or streams ordered by events).
  */
 #ifndef RAE_H_
 #define RAE_H_
