@@ -199,7 +199,11 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
           used = false;
         }
         const int64_t w = units[u].w;
-        const int64_t take = std::min<int64_t>(rb, std::max<int64_t>((cap - ovh) / w, 1));
+        // w is 1 or 2 in practice: avoid a 64-bit division in this innermost loop (the binary
+        // search runs it a dozen times per plan)
+        const int64_t room = cap - ovh;
+        const int64_t fit = w == 1 ? room : (w == 2 ? (room >> 1) : room / w);
+        const int64_t take = std::min<int64_t>(rb, std::max<int64_t>(fit, 1));
         if (emit) {
           pieces.push_back({int32_t(u), int32_t(s), int32_t(take), int32_t(c)});
           npieces[u] += 1;
@@ -220,7 +224,9 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
     pieces.clear();
     std::fill(npieces.begin(), npieces.end(), 0);
     int64_t lo = std::max<int64_t>(ceil_div(total, grid), ovh + 1);
-    int64_t hi = lo;
+    // Bracket: a CTA's fill falls short of its capacity by less than one unit's cost, so the
+    // even share plus the largest unit (and an overhead) almost always fits; double if not.
+    int64_t hi = lo + maxc + ovh;
     while (greedy(hi, false) > grid) hi *= 2;
     while (lo < hi) {
       const int64_t mid = lo + (hi - lo) / 2;
