@@ -164,11 +164,20 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
         gtotal[u] = gcost[gi].second;
       }
     }
-    std::stable_sort(order.begin(), order.end(), [&](int64_t a, int64_t b) {
-      if (gtotal[a] != gtotal[b]) return gtotal[a] > gtotal[b];
-      if (units[a].group != units[b].group) return units[a].group < units[b].group;
-      return cost[a] > cost[b];
+    // (descending group total, group, descending cost, index): the index makes the order
+    // total, so a plain sort gives the stable order
+    struct Key {
+      int64_t gt, grp, c, u;
+    };
+    std::vector<Key> keys(nu);
+    for (int64_t u = 0; u < nu; ++u) keys[u] = {-gtotal[u], units[u].group, -cost[u], u};
+    std::sort(keys.begin(), keys.end(), [](const Key& a, const Key& b) {
+      if (a.gt != b.gt) return a.gt < b.gt;
+      if (a.grp != b.grp) return a.grp < b.grp;
+      if (a.c != b.c) return a.c < b.c;
+      return a.u < b.u;
     });
+    for (int64_t i = 0; i < nu; ++i) order[i] = keys[i].u;
     const int32_t ctas = int32_t(std::min<int64_t>(grid, nu));
     using Load = std::pair<int64_t, int32_t>;
     std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
@@ -180,8 +189,15 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
       npieces[u] = 1;
       heap.push({l.first + cost[u], l.second});
     }
-    std::stable_sort(pieces.begin(), pieces.end(),
-                     [](const Piece& a, const Piece& b) { return a.cta < b.cta; });
+    // group by CTA, keeping each CTA's pieces in assignment order (a stable counting sort)
+    {
+      std::vector<int64_t> start(size_t(ctas) + 1, 0);
+      for (const Piece& pc : pieces) ++start[size_t(pc.cta) + 1];
+      for (int32_t c = 0; c < ctas; ++c) start[size_t(c) + 1] += start[size_t(c)];
+      std::vector<Piece> sorted(pieces.size());
+      for (const Piece& pc : pieces) sorted[size_t(start[size_t(pc.cta)]++)] = pc;
+      pieces.swap(sorted);
+    }
     num_ctas = ctas;
   };
 
