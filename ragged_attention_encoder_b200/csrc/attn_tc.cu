@@ -94,11 +94,12 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
 template <int D>
 __device__ __forceinline__ void mma_s(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr,
                                       uint32_t idesc) {
+  const uint64_t qd = smem_desc_sw128(q_addr, 16, 1024);
+  const uint64_t kd = smem_desc_sw128(k_addr, 16, 1024);
 #pragma unroll
   for (int ks = 0; ks < D / 16; ++ks) {
     const uint32_t off = (ks >> 2) * kChunkBytes + (ks & 3) * 32;
-    umma_ss(d_tmem, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-            idesc, ks > 0 ? 1u : 0u);
+    umma_ss(d_tmem, qd + (off >> 4), kd + (off >> 4), idesc, ks > 0 ? 1u : 0u);
   }
 }
 
@@ -106,10 +107,11 @@ __device__ __forceinline__ void mma_s(uint32_t d_tmem, uint32_t q_addr, uint32_t
 template <int D>
 __device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_addr,
                                        uint32_t idesc, bool first) {
+  const uint64_t vd = smem_desc_sw128(v_addr, kChunkBytes, 1024);
 #pragma unroll
   for (int ks = 0; ks < kTcBlockKeys / 16; ++ks)
-    umma_ts(o_tmem, p_tmem + ks * 8, smem_desc_sw128(v_addr + ks * 16 * 128, kChunkBytes, 1024),
-            idesc, (ks > 0 || !first) ? 1u : 0u);
+    umma_ts(o_tmem, p_tmem + ks * 8, vd + uint64_t((ks * 16 * 128) >> 4), idesc,
+            (ks > 0 || !first) ? 1u : 0u);
 }
 
 // O row *= f, 16 columns at a time (rare: only when a row's maximum grew by more than 2^8).
