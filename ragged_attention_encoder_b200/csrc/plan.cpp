@@ -184,15 +184,31 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
     });
     for (int64_t i = 0; i < nu; ++i) order[i] = keys[i].u;
     const int32_t ctas = int32_t(std::min<int64_t>(grid, nu));
+    // Min-heap of (load, cta): each unit goes to the least-loaded CTA (lowest index on ties),
+    // whose load then grows -- one sift-down per unit instead of a pop and a push.
     using Load = std::pair<int64_t, int32_t>;
-    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
-    for (int32_t c = 0; c < ctas; ++c) heap.push({0, c});
+    std::vector<Load> heap;
+    heap.resize(static_cast<size_t>(ctas));
+    for (int32_t c = 0; c < ctas; ++c) heap[size_t(c)] = {0, c};   // already a heap
+    pieces.reserve(size_t(nu));
     for (int64_t u : order) {
-      Load l = heap.top();
-      heap.pop();
-      pieces.push_back({int32_t(u), 0, int32_t(nb[u]), l.second});
+      Load& top = heap[0];
+      pieces.push_back({int32_t(u), 0, int32_t(nb[u]), top.second});
       npieces[u] = 1;
-      heap.push({l.first + cost[u], l.second});
+      top.first += cost[u];
+      const Load moved = top;
+      size_t i = 0;
+      while (true) {
+        const size_t l = 2 * i + 1, r = l + 1;
+        size_t m = i;
+        const Load* best = &moved;
+        if (l < heap.size() && heap[l] < *best) { m = l; best = &heap[l]; }
+        if (r < heap.size() && heap[r] < *best) { m = r; best = &heap[r]; }
+        if (m == i) break;
+        heap[i] = heap[m];
+        i = m;
+      }
+      heap[i] = moved;
     }
     // group by CTA, keeping each CTA's pieces in assignment order (a stable counting sort)
     {
@@ -474,6 +490,7 @@ int build_ragged_plan(const rae_config& cfg, const int32_t* cu_q, const int32_t*
   const int32_t tile_tok = kTcRows / g;
   const int32_t tok_per_unit = 2 * tile_tok;   // two 128-row query tiles per unit
   std::vector<Unit> units;
+  units.reserve(size_t(num_spans) * size_t(cfg.num_kv_heads) * 4);
   for (int32_t s = 0; s < num_spans; ++s) {
     const int32_t lq = cu_q[s + 1] - cu_q[s];
     const int32_t lk = kv[s + 1] - kv[s];
