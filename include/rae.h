@@ -108,7 +108,9 @@ typedef struct rae_plan {
   int32_t off_b;
   int32_t off_c;
   int32_t off_d;
-  int32_t reserved;
+  int32_t kv_extent;         /* what a run's K/V must hold: 1 + the largest page id listed
+                                (paged plans: the run's num_pages must be at least this) or
+                                the key tokens the spans read (ragged plans: total_kv) */
 } rae_plan;
 
 /* Creates a context on the current CUDA device.  Fails with RAE_ERR_UNSUPPORTED on a GPU
@@ -217,12 +219,6 @@ int rae_plan_paged(rae_ctx* ctx, int32_t slot, const int32_t* qo_indptr,
                    void* stream, rae_plan* out);
 
 /*
- * Plan of cacheless ragged attention (RaggedBlockCausalAttnManager / RaggedCrossAttnManager).
- * Host int32 arrays cu_q [S+1] and cu_kv [S+1] (NULL: self-attention, keys are the query
- * span).  block_size > 0: block-causal, local position i sees j iff j / bs <= i / bs (blocks
- * counted from each span's start); block_size == 0: every key of the span is visible.
- */
-/*
  * Plan of paged causal self-attention (page "mstar.engine.resources.attn.config",
  * AttentionStep with causal=True): the same arrays as rae_plan_paged, where the
  * qo_indptr[b+1] - qo_indptr[b] queries of request b are the last tokens of its kv_len[b]
@@ -234,6 +230,12 @@ int rae_plan_paged_causal(rae_ctx* ctx, int32_t slot, const int32_t* qo_indptr,
                           const int32_t* kv_len, int32_t batch, int32_t num_pages,
                           void* workspace, void* stream, rae_plan* out);
 
+/*
+ * Plan of cacheless ragged attention (RaggedBlockCausalAttnManager / RaggedCrossAttnManager).
+ * Host int32 arrays cu_q [S+1] and cu_kv [S+1] (NULL: self-attention, keys are the query
+ * span).  block_size > 0: block-causal, local position i sees j iff j / bs <= i / bs (blocks
+ * counted from each span's start); block_size == 0: every key of the span is visible.
+ */
 int rae_plan_ragged(rae_ctx* ctx, int32_t slot, const int32_t* cu_q, const int32_t* cu_kv,
                     int32_t num_spans, int32_t block_size, void* workspace, void* stream,
                     rae_plan* out);
@@ -241,14 +243,19 @@ int rae_plan_ragged(rae_ctx* ctx, int32_t slot, const int32_t* cu_q, const int32
 /*
  * One layer's paged cross-attention (FlashInferCrossManager.run): reads q [total_q, Hq, d],
  * k_pool, v_pool (device, bf16; never written) and writes out [total_q, Hq, d] (device, bf16).
- * sm_scale <= 0 selects 1/sqrt(head_dim).  The plan must come from rae_plan_paged on this
- * context with the same workspace, and its slot must not have been re-planned since.
+ * sm_scale <= 0 selects 1/sqrt(head_dim).  The plan must come from rae_plan_paged (or
+ * rae_plan_paged_causal) on this context with the same workspace, and its slot must not have
+ * been re-planned since.  num_pages is the number of pages the pools hold; a plan that lists
+ * a page id >= num_pages (num_pages < plan->kv_extent) is rejected with RAE_ERR_INVALID_ARG
+ * before anything is launched.
  */
 int rae_run_paged(rae_ctx* ctx, const rae_plan* plan, const void* q, const void* k_pool,
                   const void* v_pool, int32_t num_pages, void* out, float sm_scale,
                   void* workspace, void* stream);
 
-/* One layer's ragged attention: q [cu_q[S], Hq, d], k, v [cu_kv[S], Hkv, d] -> out. */
+/* One layer's ragged attention: q [cu_q[S], Hq, d], k, v [cu_kv[S], Hkv, d] -> out (device,
+ * bf16).  total_kv is the number of key tokens k and v hold; fewer than the plan's spans read
+ * (total_kv < plan->kv_extent) is rejected with RAE_ERR_INVALID_ARG before any launch. */
 int rae_run_ragged(rae_ctx* ctx, const rae_plan* plan, const void* q, const void* k,
                    const void* v, int32_t total_kv, void* out, float sm_scale, void* workspace,
                    void* stream);

@@ -66,7 +66,7 @@ class RaePlan(ctypes.Structure):
         ("off_b", i32),
         ("off_c", i32),
         ("off_d", i32),
-        ("reserved", i32),
+        ("kv_extent", i32),
     ]
 
 

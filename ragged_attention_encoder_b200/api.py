@@ -49,6 +49,16 @@ def _ptr32(a: np.ndarray):
     return a.ctypes.data_as(_lib.P32)
 
 
+def _shape(t: torch.Tensor, name: str, shape) -> None:
+    """Raises unless t has len(shape) dimensions matching shape (None: any extent).  The
+    library reads and writes whole rows of these buffers, so a short one must not reach it."""
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a tensor")
+    if t.dim() != len(shape) or any(e is not None and t.shape[i] != e for i, e in enumerate(shape)):
+        want = ", ".join("*" if e is None else str(e) for e in shape)
+        raise ValueError(f"{name} must have shape [{want}], got {list(t.shape)}")
+
+
 def _dev(t: torch.Tensor, name: str, dtype=torch.bfloat16) -> int:
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -132,6 +142,13 @@ class Context:
             msg = self._lib.rae_last_error(self._h)
             _raise(st, msg.decode() if msg else "")
 
+    def _pools(self, k_pool, v_pool):
+        _shape(k_pool, "k_pool", (None, self.num_kv_heads, self.page_size, self.head_dim))
+        _shape(v_pool, "v_pool", tuple(k_pool.shape))
+
+    def _tokens(self, t, name, rows, heads):
+        _shape(t, name, (rows, heads, self.head_dim))
+
     def _slot(self, slot):
         if slot is None:
             slot = self._next_slot
@@ -181,6 +198,10 @@ class Context:
         batch = int(cu.shape[0] - 1)
         if ip.shape[0] != batch + 1:
             raise ValueError("page_indptr must have batch + 1 entries")
+        n = int(cu[-1]) if batch > 0 else 0
+        self._tokens(k_src, "k_src", n, self.num_kv_heads)
+        self._tokens(v_src, "v_src", n, self.num_kv_heads)
+        self._pools(k_pool, v_pool)
         self._check(self._lib.rae_write_context(
             self._h, _dev(k_src, "k_src"), _dev(v_src, "v_src"), _ptr32(cu), _ptr32(ip),
             _ptr32(ix) if ix.size else None, batch, _dev(k_pool, "k_pool"),
@@ -204,6 +225,7 @@ class Context:
             raise ValueError("hidden must be [tokens, H] and w_k, w_v [num_kv_heads * head_dim, H]")
         if hidden.shape[0] != int(cu[-1]):
             raise ValueError("hidden must have cu_enc[-1] rows")
+        self._pools(k_pool, v_pool)
         for b, name in ((b_k, "b_k"), (b_v, "b_v")):
             if b is not None and tuple(b.shape) != (n_out,):
                 raise ValueError(f"{name} must have num_kv_heads * head_dim entries")
@@ -225,6 +247,10 @@ class Context:
         batch = int(kl.shape[0])
         if ap.shape[0] != batch + 1 or ip.shape[0] != batch + 1:
             raise ValueError("append_indptr and kv_page_indptr must have batch + 1 entries")
+        n = int(ap[-1]) if batch > 0 else 0
+        self._tokens(k_new, "k_new", n, self.num_kv_heads)
+        self._tokens(v_new, "v_new", n, self.num_kv_heads)
+        self._pools(k_pool, v_pool)
         self._check(self._lib.rae_append_kv(
             self._h, _dev(k_new, "k_new"), _dev(v_new, "v_new"), _ptr32(ap), _ptr32(ip),
             _ptr32(ix) if ix.size else None, _ptr32(kl) if kl.size else None, batch,
@@ -266,8 +292,11 @@ class Context:
         return Plan(raw, "ragged", total_kv=total_kv)
 
     def run_paged(self, plan: Plan, q, k_pool, v_pool, out=None, sm_scale: float = 0.0):
+        self._tokens(q, "q", plan.total_q, self.num_qo_heads)
+        self._pools(k_pool, v_pool)
         if out is None:
             out = torch.empty_like(q)
+        _shape(out, "out", tuple(q.shape))
         self._check(self._lib.rae_run_paged(
             self._h, ctypes.byref(plan.raw), _dev(q, "q"), _dev(k_pool, "k_pool"),
             _dev(v_pool, "v_pool"), int(k_pool.shape[0]), _dev(out, "out"), float(sm_scale),
@@ -275,8 +304,12 @@ class Context:
         return out
 
     def run_ragged(self, plan: Plan, q, k, v, out=None, sm_scale: float = 0.0):
+        self._tokens(q, "q", plan.total_q, self.num_qo_heads)
+        self._tokens(k, "k", None, self.num_kv_heads)
+        _shape(v, "v", tuple(k.shape))
         if out is None:
             out = torch.empty_like(q)
+        _shape(out, "out", tuple(q.shape))
         self._check(self._lib.rae_run_ragged(
             self._h, ctypes.byref(plan.raw), _dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
             int(k.shape[0]), _dev(out, "out"), float(sm_scale), self.workspace.data_ptr(),

@@ -498,6 +498,10 @@ int rae_run_paged(rae_ctx* ctx, const rae_plan* plan, const void* q, const void*
   if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
     return set_err(ctx, RAE_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
   if (num_pages <= 0) return set_err(ctx, RAE_ERR_INVALID_ARG, "num_pages must be positive");
+  if (num_pages < plan->kv_extent)
+    return set_err(ctx, RAE_ERR_INVALID_ARG,
+                   "the plan lists page " + std::to_string(plan->kv_extent - 1) + " but the pools hold " +
+                       std::to_string(num_pages) + " pages");
   const rae_config& c = ctx->cfg;
   const Geometry geo = geometry(c);
   const DevPlan dp = dev_plan(ctx, plan, workspace);
@@ -548,7 +552,10 @@ int rae_run_ragged(rae_ctx* ctx, const rae_plan* plan, const void* q, const void
     return set_err(ctx, RAE_ERR_INVALID_ARG, "NULL device pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return set_err(ctx, RAE_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
-  if (total_kv < 0) return set_err(ctx, RAE_ERR_INVALID_ARG, "total_kv < 0");
+  if (total_kv < plan->kv_extent)
+    return set_err(ctx, RAE_ERR_INVALID_ARG,
+                   "the plan reads " + std::to_string(plan->kv_extent) + " key tokens but k and v hold " +
+                       std::to_string(total_kv));
   const rae_config& c = ctx->cfg;
   const Geometry geo = geometry(c);
   const DevPlan dp = dev_plan(ctx, plan, workspace);

@@ -395,11 +395,14 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
   if (num_pages < 0) return fail(err, RAE_ERR_INVALID_ARG, "num_pages < 0");
   if (int64_t(num_pages) * cfg.num_kv_heads * cfg.page_size >= (int64_t(1) << 31))
     return fail(err, RAE_ERR_CAPACITY, "pool rows overflow int32");
-  for (int32_t i = 0; i < nnz; ++i)
+  int32_t page_extent = 0;   // 1 + the largest page id listed: the pool a run must hold
+  for (int32_t i = 0; i < nnz; ++i) {
     if (kv_page_indices[i] < 0 || kv_page_indices[i] >= num_pages)
       return fail(err, RAE_ERR_INVALID_ARG,
                   "page id " + std::to_string(kv_page_indices[i]) + " at " + std::to_string(i) +
                       " outside [0, num_pages)");
+    page_extent = std::max(page_extent, kv_page_indices[i] + 1);
+  }
   for (int32_t b = 0; b < batch; ++b) {
     if (kv_len[b] < 0) return fail(err, RAE_ERR_INVALID_ARG, "kv_len < 0");
     int64_t need = ceil_div(kv_len[b], cfg.page_size);
@@ -450,6 +453,7 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
   out->batch = batch;
   out->total_q = total_q;
   out->block_size = causal ? 1 : 0;
+  out->kv_extent = page_extent;
   int32_t rows_max = 0;
   for (const Unit& u : units) rows_max = std::max(rows_max, u.rows);
   if (swap) rows_max = swap_n;   // the row count the swapped kernel is instantiated for
@@ -516,6 +520,7 @@ int build_ragged_plan(const rae_config& cfg, const int32_t* cu_q, const int32_t*
   out->batch = num_spans;
   out->total_q = total_q;
   out->block_size = block_size;
+  out->kv_extent = kv[num_spans];
   out->rows_max = 0;
   for (const Unit& u : units) out->rows_max = std::max(out->rows_max, u.rows);
   Schedule sc;

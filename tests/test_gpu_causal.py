@@ -78,9 +78,10 @@ def test_append_rejects_more_tokens_than_the_stream():
     case = _stream_case(301, [2], [5], 2, 2, 64, 16)
     ctx = Context(2, 2, 64, 16)
     kp = inputs.nan_pool(case.num_pages, 2, 16, 64, "cuda")
+    k_new = torch.zeros(6, 2, 64, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(ValueError, match="more tokens"):
-        ctx.append_kv(case.k_ctx.cuda(), case.v_ctx.cuda(), [0, 6], case.kv_page_indptr,
-                      case.kv_page_indices, case.kv_len, kp, kp.clone())
+        ctx.append_kv(k_new, k_new, [0, 6], case.kv_page_indptr, case.kv_page_indices,
+                      case.kv_len, kp, kp.clone())
 
 
 @pytest.mark.parametrize("hq,hkv,d,P,q_lens,kind", [

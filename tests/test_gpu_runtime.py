@@ -73,6 +73,33 @@ def test_bad_tensors_are_rejected_before_launch():
         Context(8, 3, 64, 16)
 
 
+def test_buffers_smaller_than_the_plan_are_rejected_before_launch():
+    """The pools must hold every page the plan lists, k / v every key its spans read, and q /
+    out exactly the plan's query rows; nothing is launched otherwise."""
+    c = _case(214)
+    ctx = Context(8, 2, 64, 16)
+    kp, vp = gpu_pools(c, ctx)
+    plan = ctx.plan_paged(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages)
+    extent = int(np.max(c.kv_page_indices)) + 1
+    assert plan.raw.kv_extent == extent
+    with pytest.raises(ValueError, match="pools hold"):
+        ctx.run_paged(plan, c.q.cuda(), kp[:extent - 1].contiguous(), vp[:extent - 1].contiguous())
+    with pytest.raises(ValueError, match="shape"):
+        ctx.run_paged(plan, c.q.cuda()[1:].contiguous(), kp, vp)
+    with pytest.raises(ValueError, match="shape"):
+        ctx.run_paged(plan, c.q.cuda(), kp, vp, torch.empty_like(c.q.cuda())[:, :1].contiguous())
+    with pytest.raises(ValueError, match="shape"):
+        ctx.run_paged(plan, c.q.cuda(), kp, vp[:, :1].contiguous())
+    rp = ctx.plan_ragged([0, 40, 100], [0, 30, 70], 0)
+    assert rp.raw.kv_extent == 70
+    q = torch.zeros(100, 8, 64, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(69, 2, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError, match="key tokens"):
+        ctx.run_ragged(rp, q, k, k.clone())
+    torch.cuda.synchronize()
+    ctx.check_device_status()
+
+
 def test_status_word_is_clear_after_normal_runs():
     c = _case(213, qmax=20)
     ctx = Context(8, 2, 64, 16)

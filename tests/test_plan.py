@@ -130,6 +130,8 @@ def test_paged_plan_covers_each_pair_once(seed, hq, hkv, d, P):
                 assert np.all(keys == 1)
     assert not cover, "tiles cover rows that do not exist"
     _check_merge(p, g, hq)
+    # the pool a run must hold: every listed page id below it
+    assert p["raw"].kv_extent == (int(indices.max()) + 1 if indices.size else 0)
 
 
 @pytest.mark.parametrize("seed", range(4))
@@ -163,6 +165,7 @@ def test_ragged_plan_covers_each_visible_pair_once(seed, bs, hq, hkv):
                 assert np.all(keys <= 1)
     assert not cover
     _check_merge(p, g, hq)
+    assert p["raw"].kv_extent == int(cu_k[-1])       # key tokens a run's k and v must hold
 
 
 def test_plan_is_deterministic():
@@ -308,6 +311,21 @@ def test_causal_plan_trims_key_ranges_to_the_last_query():
                         num_kv_heads=2, head_dim=128, page_size=16, causal=True, num_sms=1)
     ends = sorted({(int(r[2]), int(r[5])) for r in p["tiles"]})
     assert ends == [(0, 1064), (64, 1128)]
+
+
+def test_binding_rejects_buffers_of_the_wrong_shape():
+    """The binding checks every device buffer's shape against the call before the library
+    sees its pointer (the kernels read and write whole rows)."""
+    import torch
+    from ragged_attention_encoder_b200.api import _shape
+    t = torch.zeros(5, 4, 64)
+    _shape(t, "q", (5, 4, 64))
+    _shape(t, "q", (None, 4, 64))
+    for bad in [(4, 4, 64), (5, 2, 64), (5, 4, 128), (5, 4), (None, 4, 64, 1)]:
+        with pytest.raises(ValueError, match="shape"):
+            _shape(t, "q", bad)
+    with pytest.raises(ValueError, match="tensor"):
+        _shape(None, "q", (5, 4, 64))
 
 
 def test_missing_library_fails_loudly():
