@@ -55,7 +55,7 @@ def test_plan_kind_must_match_run():
     c = _case(211)
     ctx = Context(8, 2, 64, 16)
     kp, vp = gpu_pools(c, ctx)
-    rp = ctx.plan_ragged([0, 4], None, 0)
+    rp = ctx.plan_ragged([0, int(c.q.shape[0])], None, 0)   # same query rows: only the kind differs
     with pytest.raises(ValueError, match="kind"):
         ctx.run_paged(rp, c.q.cuda(), kp, vp)
 
