@@ -36,9 +36,16 @@ int64_t align4(int64_t w) { return (w + 3) & ~int64_t(3); }
 
 struct Unit {
   int32_t req, kvh, q0, qn, nkeys, rows;
-  int32_t w;       // work per key block: the number of 128-row query tiles the unit holds
+  int32_t w;       // cost of one key block (the scheduler's unit; see tc_block_cost)
   int64_t group;   // units of one group read the same K/V (one request or span, one KV head)
 };
+
+// Cost of one 128-key block of a tensor-core unit, in 1/16 of a block step.  The kernel is
+// bound by the hand-off between its MMA and softmax warps, not by tensor throughput: a block
+// takes about as long with one 128-row query tile as with two (measured 1.05x for two full
+// tiles against one), so a unit's cost follows its key blocks, not its rows.
+constexpr int32_t kTcStep = 16;
+int32_t tc_block_cost(int32_t tiles) { return tiles > 1 ? kTcStep + 1 : kTcStep; }
 
 struct Piece {
   int32_t unit, blk0, nblk, cta;
@@ -128,7 +135,8 @@ int emit_image(const Schedule& sc, const int32_t* a, int64_t na, const int32_t* 
 }
 
 // Schedules units over the grid: tiles, CTA pointers and merge rows.
-//   blk: keys per block; ovh: per-tile overhead in blocks; g: query heads per KV head.
+//   blk: keys per block; ovh: per-tile overhead in the units of Unit::w; g: query heads per
+//   KV head.
 //   lpt_factor: whole units are scheduled longest-first when every CTA's share is at least
 //   lpt_factor times the largest unit; otherwise the balanced contiguous partition is used.
 int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units, int32_t blk,
@@ -222,7 +230,7 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
     num_ctas = ctas;
   };
 
-  // Greedy fill of CTAs with capacity q (blocks + overhead per piece), in unit order;
+  // Greedy fill of CTAs with capacity q (block costs + overhead per piece), in unit order;
   // returns the CTAs used, and the pieces when `emit` is set.
   auto greedy = [&](int64_t q, bool emit) -> int64_t {
     int64_t c = 0, cap = q;
@@ -236,10 +244,12 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
           used = false;
         }
         const int64_t w = units[u].w;
-        // w is 1 or 2 in practice: avoid a 64-bit division in this innermost loop (the binary
-        // search runs it a dozen times per plan)
+        // room >= 1; a 32-bit division where it fits (the binary search runs this innermost
+        // loop a dozen times per plan)
         const int64_t room = cap - ovh;
-        const int64_t fit = w == 1 ? room : (w == 2 ? (room >> 1) : room / w);
+        const int64_t fit = w == 1 ? room
+                            : room < (int64_t(1) << 32) ? int64_t(uint32_t(room) / uint32_t(w))
+                                                        : room / w;
         const int64_t take = std::min<int64_t>(rb, std::max<int64_t>(fit, 1));
         if (emit) {
           pieces.push_back({int32_t(u), int32_t(s), int32_t(take), int32_t(c)});
@@ -444,7 +454,7 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
         // keys; no row of the unit sees more
         u.nkeys = causal ? kv_len[b] - qlen + t + u.qn : kv_len[b];
         u.rows = u.qn * g;
-        u.w = (simt || swap) ? 1 : ceil_div32(u.qn, tile_tok);
+        u.w = (simt || swap) ? 1 : tc_block_cost(ceil_div32(u.qn, tile_tok));
         u.group = int64_t(b) * cfg.num_kv_heads + h;
         units.push_back(u);
       }
@@ -462,7 +472,7 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
   // The decode kernel is HBM bound and short: an even split of the bytes over the grid
   // matters more than the small merge it costs.
   rc = simt ? schedule(cfg, kind, units, kSimtChunkKeys, 2, g, 64, &sc, err)
-            : schedule(cfg, kind, units, kTcBlockKeys, 1, g, 4, &sc, err);
+            : schedule(cfg, kind, units, kTcBlockKeys, swap ? 1 : kTcStep, g, 4, &sc, err);
   if (rc) return rc;
   rc = emit_image(sc, qo_indptr, batch + 1, kv_len, batch, kv_page_indptr, batch + 1,
                   kv_page_indices, nnz, image, image_words, out, err);
@@ -512,7 +522,7 @@ int build_ragged_plan(const rae_config& cfg, const int32_t* cu_q, const int32_t*
         }
         u.nkeys = int32_t(lim);
         u.rows = u.qn * g;
-        u.w = ceil_div32(u.qn, tile_tok);
+        u.w = tc_block_cost(ceil_div32(u.qn, tile_tok));
         u.group = int64_t(s) * cfg.num_kv_heads + h;
         units.push_back(u);
       }
@@ -524,7 +534,7 @@ int build_ragged_plan(const rae_config& cfg, const int32_t* cu_q, const int32_t*
   out->rows_max = 0;
   for (const Unit& u : units) out->rows_max = std::max(out->rows_max, u.rows);
   Schedule sc;
-  rc = schedule(cfg, kKindTcRagged, units, kTcBlockKeys, 1, g, 4, &sc, err);
+  rc = schedule(cfg, kKindTcRagged, units, kTcBlockKeys, kTcStep, g, 4, &sc, err);
   if (rc) return rc;
   rc = emit_image(sc, cu_q, num_spans + 1, kv, num_spans + 1, nullptr, 0, nullptr, 0, image,
                   image_words, out, err);
