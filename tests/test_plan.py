@@ -313,6 +313,24 @@ def test_causal_plan_trims_key_ranges_to_the_last_query():
     assert ends == [(0, 1064), (64, 1128)]
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_tensor_core_plan_balances_block_steps(seed):
+    """The tensor-core kernel spends about the same time on a key block whether the unit holds
+    one 128-row query tile or two, so the plan balances block steps (plus one per tile): on
+    block-causal spans of the benchmark's shape, with many one-tile span tails, the busiest
+    CTA carries at most 4 % more steps than the mean."""
+    rng = np.random.default_rng(seed)
+    lens = []
+    while sum(lens) < 65536:
+        lens.append(int(rng.integers(256, 4097)))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    p = plan_ragged_host(cu, None, 256, num_qo_heads=16, num_kv_heads=16, head_dim=128)
+    t, cp = p["tiles"], p["cta_ptr"]
+    steps = [sum(-(-(int(t[i, 5]) - int(t[i, 4])) // 128) + 1 for i in range(cp[c], cp[c + 1]))
+             for c in range(p["raw"].num_ctas)]
+    assert max(steps) <= 1.04 * np.mean(steps), (max(steps), np.mean(steps))
+
+
 def test_binding_rejects_buffers_of_the_wrong_shape():
     """The binding checks every device buffer's shape against the call before the library
     sees its pointer (the kernels read and write whole rows)."""
