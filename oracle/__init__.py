@@ -19,7 +19,6 @@ from .attention import (  # noqa: F401
     as_f64,
     attention_rows,
     block_causal_visible,
-    block_causal_key_limit,
     causal_append_visible,
     context_write,
     gather_paged_kv,

@@ -134,11 +134,6 @@ def block_causal_visible(length: int, block_size: int) -> np.ndarray:
     return (j // block_size) <= (i // block_size)
 
 
-def block_causal_key_limit(length: int, block_size: int) -> np.ndarray:
-    """Number of visible keys of each position of a span, counted from the mask above."""
-    return block_causal_visible(length, block_size).sum(axis=1)
-
-
 def gather_paged_kv(pool, page_indptr, page_indices, request: int, kv_len: int) -> np.ndarray:
     """Logical K (or V) rows [kv_len, Hkv, d] of one request, read through its page list."""
     page_size = pool.shape[2]

@@ -224,6 +224,26 @@ def test_context_write_places_every_token_and_nothing_else():
     assert touched.sum() == case.kv_len.sum()
 
 
+def test_gather_reads_back_what_the_context_write_placed():
+    """Reading a request's keys through its page list returns, in order, the rows the
+    context write (pinned above against a page-walking enumeration) placed: a transposed
+    page/slot index or a page list read out of order would return other rows."""
+    case = inputs.paged_case(23, q_lens=[1, 1, 1], ctx_lens=[5, 16, 50], num_qo_heads=4,
+                             num_kv_heads=2, head_dim=8, page_size=16, pool_pages=10)
+    kp, vp = _oracle_pools(case)
+    for b in range(case.batch):
+        c0, c1 = int(case.cu_enc[b]), int(case.cu_enc[b + 1])
+        for pool, src in ((kp, case.k_ctx), (vp, case.v_ctx)):
+            got = oracle.gather_paged_kv(pool, case.kv_page_indptr, case.kv_page_indices, b,
+                                         int(case.kv_len[b]))
+            assert got.shape == (c1 - c0, 2, 8)
+            assert np.array_equal(got, src[c0:c1].double().numpy())
+    # a prefix of the stream reads the same first rows
+    got = oracle.gather_paged_kv(kp, case.kv_page_indptr, case.kv_page_indices, 2, 17)
+    assert np.array_equal(got, case.k_ctx[int(case.cu_enc[2]):int(case.cu_enc[2]) + 17]
+                          .double().numpy())
+
+
 def test_page_permutation_invariance():
     case = inputs.paged_case(22, q_lens=[2, 3], ctx_lens=[20, 45], num_qo_heads=4, num_kv_heads=2,
                              head_dim=16, page_size=16, pool_pages=12)
@@ -378,6 +398,23 @@ def test_paged_causal_prefill_is_sdpa_causal(hq, hkv):
         assert np.allclose(out[q0:q1], ref, atol=1e-12, rtol=0)
 
 
+@pytest.mark.parametrize("qlen,kv_len", [(1, 1), (1, 9), (4, 4), (3, 10), (7, 7), (5, 6)])
+def test_causal_append_mask_brute_force(qlen, kv_len):
+    """Walk the stream: its last qlen tokens are the queries, each sees every token up to
+    and including its own position.  qlen == kv_len is the textbook lower triangle."""
+    expect = np.zeros((qlen, kv_len), dtype=bool)
+    for i in range(qlen):
+        own = kv_len - qlen + i             # stream position of query i
+        for j in range(kv_len):
+            expect[i, j] = j <= own
+    got = oracle.causal_append_visible(qlen, kv_len)
+    assert np.array_equal(got, expect)
+    if qlen == kv_len:
+        assert np.array_equal(got, np.tril(np.ones((qlen, qlen), bool)))
+    if qlen == 1:
+        assert got.all()
+
+
 def test_paged_causal_query_sees_the_stream_up_to_itself():
     """Query i of a step is the stream's token kv_len - qlen + i: its result equals
     cross-attention (pinned to SDPA) of that query over the stream cut just after it."""
@@ -509,3 +546,16 @@ def test_projection_is_affine_and_zero_weights_give_the_bias():
     zero = torch.zeros_like(wk)
     k0, v0 = oracle.project_kv(x1, zero, bk, zero, None, hkv, d)
     assert np.array_equal(k0, np.broadcast_to(b, k0.shape)) and not np.any(v0)
+
+
+def test_every_exported_oracle_function_has_a_pin_here():
+    """Every function the oracle exports is called by at least one test of this file."""
+    import inspect
+    import re
+    src = inspect.getsource(inspect.getmodule(test_every_exported_oracle_function_has_a_pin_here))
+    body = src.split("def test_every_exported_oracle_function_has_a_pin_here")[0]
+    exported = [n for n, f in vars(oracle).items()
+                if callable(f) and not n.startswith("_") and getattr(f, "__module__", "").startswith("oracle")]
+    assert exported
+    missing = [n for n in exported if not re.search(r"oracle\." + n + r"\(", body)]
+    assert not missing, f"oracle functions without a pin: {missing}"
