@@ -120,7 +120,8 @@ int rae_create(rae_ctx** out, const rae_config* cfg);
 /* Waits for the context's pending staging copies and frees its host resources. */
 int rae_destroy(rae_ctx* ctx);
 
-/* Message for the last failing call on ctx (a static string when ctx is NULL). */
+/* Message for the last failing call on ctx.  With ctx NULL: the message of the calling
+ * thread's last failing rae_write_context_noalloc call ("no context" if there was none). */
 const char* rae_last_error(const rae_ctx* ctx);
 
 /* Bytes of device workspace the caller must allocate (256-byte aligned) and pass to every
@@ -158,9 +159,13 @@ int rae_write_context(rae_ctx* ctx, const void* k_src, const void* v_src, const 
  *     before any device work.
  *   - The first call on a device looks up the array's device address (with that device
  *     current); make that first call before any stream capture.
+ *   - The list reaches the device array by a copy from one host array of the library, which
+ *     the next call rewrites.  While `stream` is capturing, the call therefore enqueues
+ *     nothing and returns RAE_ERR_UNSUPPORTED.
  *   - All calls share the one array, which keeps the last call's list: calls that overlap on
  *     the GPU (different streams, not ordered) race on it and must be serialised by the caller.
  *   - The host arrays may be reused as soon as the call returns.
+ *   - A failing call leaves its message for rae_last_error(NULL) on the calling thread.
  */
 int rae_write_context_noalloc(const void* k_src, const void* v_src, const int32_t* cu_enc,
                               const int32_t* page_indptr, const int32_t* page_indices,

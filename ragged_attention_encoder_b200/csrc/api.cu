@@ -264,7 +264,7 @@ int rae_destroy(rae_ctx* ctx) {
 }
 
 const char* rae_last_error(const rae_ctx* ctx) {
-  if (!ctx) return "no context";
+  if (!ctx) return rae::noalloc_last_error();
   return ctx->last_error.c_str();
 }
 

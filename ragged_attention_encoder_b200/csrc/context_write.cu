@@ -95,6 +95,23 @@ std::mutex g_noalloc_mutex;
 }  // namespace
 }  // namespace rae
 
+namespace rae {
+// Message of the calling thread's last failing rae_write_context_noalloc call (the call has
+// no context to keep it in); rae_last_error(NULL) returns it.
+thread_local std::string g_noalloc_msg;
+
+const char* noalloc_last_error() {
+  return g_noalloc_msg.empty() ? "no context" : g_noalloc_msg.c_str();
+}
+
+namespace {
+int noalloc_fail(int code, const std::string& msg) {
+  g_noalloc_msg = "rae_write_context_noalloc: " + msg;
+  return code;
+}
+}  // namespace
+}  // namespace rae
+
 extern "C" int rae_write_context_noalloc(const void* k_src, const void* v_src,
                                          const int32_t* cu_enc, const int32_t* page_indptr,
                                          const int32_t* page_indices, int32_t batch,
@@ -102,13 +119,25 @@ extern "C" int rae_write_context_noalloc(const void* k_src, const void* v_src,
                                          int32_t num_kv_heads, int32_t head_dim,
                                          int32_t page_size, void* stream) {
   using namespace rae;
-  if (!k_pool || !v_pool) return RAE_ERR_INVALID_ARG;
+  if (!k_pool || !v_pool) return noalloc_fail(RAE_ERR_INVALID_ARG, "k_pool or v_pool is NULL");
   const uintptr_t mis = reinterpret_cast<uintptr_t>(k_src) | reinterpret_cast<uintptr_t>(v_src) |
                         reinterpret_cast<uintptr_t>(k_pool) | reinterpret_cast<uintptr_t>(v_pool);
-  if (mis & 15) return RAE_ERR_INVALID_ARG;
+  if (mis & 15) return noalloc_fail(RAE_ERR_INVALID_ARG, "a device buffer is not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The page list is copied from one host array that the next call rewrites.  A copy
+  // recorded into a graph would read that array when the graph is launched, i.e. a later
+  // call's list, so the call refuses to be recorded.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess)
+    return noalloc_fail(RAE_ERR_CUDA, "cudaStreamIsCapturing failed");
+  if (cap != cudaStreamCaptureStatusNone)
+    return noalloc_fail(RAE_ERR_UNSUPPORTED,
+                        "the stream is capturing; the page list comes from a host array that "
+                        "the next call rewrites");
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return RAE_ERR_CUDA;
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return RAE_ERR_UNSUPPORTED;
+  if (cudaGetDevice(&dev) != cudaSuccess) return noalloc_fail(RAE_ERR_CUDA, "cudaGetDevice failed");
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return noalloc_fail(RAE_ERR_UNSUPPORTED, "device ordinal above " + std::to_string(kNoAllocMaxDevices - 1));
 
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
   if (!g_noalloc_dev[dev]) {
@@ -116,7 +145,8 @@ extern "C" int rae_write_context_noalloc(const void* k_src, const void* v_src,
     // stand-in, the kernel needs the address the runtime gives for this device.
     void* addr = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_items);
-    if (e != cudaSuccess || !addr) return RAE_ERR_CUDA;
+    if (e != cudaSuccess || !addr)
+      return noalloc_fail(RAE_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
     g_noalloc_dev[dev] = static_cast<WriteItem*>(addr);
   }
 
@@ -137,15 +167,19 @@ extern "C" int rae_write_context_noalloc(const void* k_src, const void* v_src,
   // device work.
   int rc = build_write_items(cfg, cu_enc, page_indptr, page_indices, nullptr, batch, num_pages,
                              g_noalloc_host, kNoAllocMaxPages, &n, &msg);
-  if (rc) return rc;
+  if (rc) {
+    if (rc == RAE_ERR_CAPACITY)
+      msg += " (at most " + std::to_string(kNoAllocMaxPages) + " page copies per call)";
+    return noalloc_fail(rc, msg);
+  }
   if (n == 0) return RAE_OK;
-  if (!k_src || !v_src) return RAE_ERR_INVALID_ARG;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!k_src || !v_src) return noalloc_fail(RAE_ERR_INVALID_ARG, "k_src or v_src is NULL");
   // From pageable host memory: the call returns once the list has been staged, so the host
   // array may be rebuilt by the next call.
   cudaError_t e = cudaMemcpyAsync(g_noalloc_dev[dev], g_noalloc_host,
                                   size_t(n) * sizeof(WriteItem), cudaMemcpyHostToDevice, st);
-  if (e != cudaSuccess) return RAE_ERR_CUDA;
+  if (e != cudaSuccess)
+    return noalloc_fail(RAE_ERR_CUDA, std::string("cudaMemcpyAsync: ") + cudaGetErrorString(e));
   Geometry geo;
   geo.hq = num_kv_heads;
   geo.hkv = num_kv_heads;
@@ -153,5 +187,7 @@ extern "C" int rae_write_context_noalloc(const void* k_src, const void* v_src,
   geo.d = head_dim;
   geo.page_size = page_size;
   e = launch_context_write(g_noalloc_dev[dev], n, k_src, v_src, k_pool, v_pool, geo, st);
-  return e == cudaSuccess ? RAE_OK : RAE_ERR_CUDA;
+  if (e != cudaSuccess)
+    return noalloc_fail(RAE_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
+  return RAE_OK;
 }

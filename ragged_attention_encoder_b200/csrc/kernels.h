@@ -90,6 +90,9 @@ struct ProjectWriteArgs {
   Geometry geo;
 };
 cudaError_t launch_project_write(const ProjectWriteArgs& args, cudaStream_t stream);
+
+// Message of the calling thread's last failing context-free call (rae_write_context_noalloc).
+const char* noalloc_last_error();
 // Output columns per tile of the projection kernel (the weight maps' box height).
 int project_write_tile_cols(int n_half);
 

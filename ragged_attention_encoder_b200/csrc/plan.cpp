@@ -246,10 +246,23 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
         const int64_t w = units[u].w;
         // room >= 1; a 32-bit division where it fits (the binary search runs this innermost
         // loop a dozen times per plan)
-        const int64_t room = cap - ovh;
-        const int64_t fit = w == 1 ? room
-                            : room < (int64_t(1) << 32) ? int64_t(uint32_t(room) / uint32_t(w))
-                                                        : room / w;
+        auto blocks_that_fit = [&]() -> int64_t {
+          const int64_t room = cap - ovh;
+          return w == 1 ? room
+                 : room < (int64_t(1) << 32) ? int64_t(uint32_t(room) / uint32_t(w))
+                                             : room / w;
+        };
+        int64_t fit = blocks_that_fit();
+        if (fit == 0 && used) {
+          // Not one block fits in what is left: start the next CTA rather than overfill
+          // this one (a block can cost more than the per-piece overhead).
+          ++c;
+          cap = q;
+          used = false;
+          fit = blocks_that_fit();
+        }
+        // An empty CTA takes at least one block even when q is too small for it; the search
+        // then finds that q needs too many CTAs.
         const int64_t take = std::min<int64_t>(rb, std::max<int64_t>(fit, 1));
         if (emit) {
           pieces.push_back({int32_t(u), int32_t(s), int32_t(take), int32_t(c)});

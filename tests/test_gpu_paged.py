@@ -190,15 +190,14 @@ def test_empty_context_gives_zero():
     assert_close(out, oracle_paged(case), what="empty ctx tc")
 
 
-@pytest.mark.parametrize("num_sms", [1, 2, 5])
+@pytest.mark.parametrize("num_sms", [2, 3, 5])
 @pytest.mark.parametrize("qmax", [1, 50])
 def test_forced_splits_agree_with_oracle_and_unsplit(num_sms, qmax):
     case = inputs.paged_case(70 + num_sms + qmax, q_lens=(1, qmax, 3), ctx_lens=(300, 3000, 3),
                              num_qo_heads=8, num_kv_heads=2, head_dim=128, page_size=32)
     ref = oracle_paged(case)
     out_split, plan, *_ = run_paged(case, num_sms=num_sms)
-    if (num_sms, qmax) in ((2, 1), (2, 50), (5, 1), (5, 50)):
-        assert plan.num_merge_rows > 0     # these seeds cut units inside their keys
+    assert plan.num_merge_rows > 0         # a small grid cuts units inside their keys
     assert_close(out_split, ref, what="split")
     out_full, plan_full, *_ = run_paged(case)
     assert_close(out_full, ref, what="unsplit")

@@ -360,3 +360,22 @@ def test_missing_library_fails_loudly():
     res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
                          timeout=120)
     assert res.stdout.strip() == "raised True", res.stdout + res.stderr
+
+
+def test_tensor_core_fill_does_not_overshoot_a_cta_by_a_block():
+    """The contiguous fill closes a CTA when not one more key block fits in its capacity, so
+    on the packed multi-token workload no CTA carries more than one block's cost above the
+    mean (block costs 16 or 17, 16 per tile)."""
+    c = inputs.workload(3)
+    p = plan_paged_host(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages,
+                        num_qo_heads=32, num_kv_heads=8, head_dim=128, page_size=16)
+    t, cp = p["tiles"], p["cta_ptr"]
+    tpt = 128 // 4
+    load = []
+    for cta in range(p["raw"].num_ctas):
+        s = 0
+        for i in range(cp[cta], cp[cta + 1]):
+            nb = -(-(int(t[i, 5]) - int(t[i, 4])) // 128)
+            s += nb * (17 if int(t[i, 3]) > tpt else 16) + 16
+        load.append(s)
+    assert max(load) <= np.mean(load) + 17, (max(load), np.mean(load))

@@ -68,5 +68,39 @@ def test_no_alloc_context_write_rejects_more_pages_than_its_array():
     vp = inputs.nan_pool(4, 1, 16, 64, "cuda")
     k = torch.zeros(16, 1, 64, dtype=torch.bfloat16, device="cuda")
     assert _noalloc(lib, case, k, k, kp, vp) == _lib.RAE_ERR_CAPACITY
+    assert b"65536" in lib.rae_last_error(None)     # the call has no context: per-thread message
     torch.cuda.synchronize()
     assert torch.all(kp.view(torch.int16) == inputs.BF16_NAN_BITS)
+
+
+def test_no_alloc_context_write_refuses_a_capturing_stream():
+    """The page list is copied from a host array that the next call rewrites, so a graph
+    replaying that copy would write a later call's pages: under capture the call enqueues
+    nothing and says why."""
+    lib = _lib.load()
+    case = inputs.paged_case(304, q_lens=[1, 1], ctx_lens=[40, 9], num_qo_heads=2,
+                             num_kv_heads=2, head_dim=64, page_size=16, pool_pages=8)
+    k, v = case.k_ctx.cuda(), case.v_ctx.cuda()
+    shape = (case.num_pages, case.num_kv_heads, case.page_size, case.head_dim)
+    kp = inputs.nan_pool(*shape, "cuda")
+    vp = inputs.nan_pool(*shape, "cuda")
+    assert _noalloc(lib, case, k, v, kp, vp) == _lib.RAE_OK     # set-up outside any capture
+    torch.cuda.synchronize()
+    kp2 = inputs.nan_pool(*shape, "cuda")
+    vp2 = inputs.nan_pool(*shape, "cuda")
+    marker = torch.zeros(1, device="cuda")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        rc = _noalloc(lib, case, k, v, kp2, vp2)
+        marker.add_(1)                           # so the captured graph is not empty
+    assert rc == _lib.RAE_ERR_UNSUPPORTED
+    assert b"capturing" in lib.rae_last_error(None)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert float(marker) == 1.0
+    assert torch.all(kp2.view(torch.int16) == inputs.BF16_NAN_BITS)
+    assert torch.all(vp2.view(torch.int16) == inputs.BF16_NAN_BITS)
+    # the stream is usable afterwards and the call works again
+    assert _noalloc(lib, case, k, v, kp2, vp2) == _lib.RAE_OK
+    torch.cuda.synchronize()
+    assert torch.equal(kp2.view(torch.int16), kp.view(torch.int16))
