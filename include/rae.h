@@ -194,6 +194,23 @@ int rae_project_write_context(rae_ctx* ctx, const void* hidden, int32_t hidden_d
                               void* v_pool, int32_t num_pages, void* workspace, void* stream);
 
 /*
+ * One tensor-parallel rank's share of the output projection (page
+ * "mstar.model.components.distributed.attention", ParallelAttention: query and KV heads are
+ * sharded over ranks -- KVConfig.shard narrows the head counts to one rank's slice -- and the
+ * only exchange of the layer is the all-reduce inside o_proj).  A rank holding query heads
+ * [h0, h0 + Hq_r) multiplies its attention output attn [m, k] (device, bf16, row-major,
+ * k = Hq_r * head_dim: the run's output of its heads) by its columns of W_o, given as
+ * w_o [n, k] (device, bf16, nn.Linear layout: row j holds W_o[j, h0*d ... (h0+Hq_r)*d)), and
+ * writes out [m, n] (device, fp32, row-major) = attn . w_o^T (+ bias [n], bf16, or NULL).
+ * The caller sums the ranks' outputs (one all-reduce); exactly one rank passes the bias.
+ * fp32 accumulation.  Requires k % 64 == 0 and n % 128 == 0 (RAE_ERR_UNSUPPORTED otherwise);
+ * every device buffer 16-byte aligned.  Asynchronous on `stream`; bounded waits report
+ * through the workspace's error word like the attention calls.
+ */
+int rae_o_proj_partial(rae_ctx* ctx, const void* attn, int32_t m, int32_t k, const void* w_o,
+                       int32_t n, const void* bias, void* out, void* workspace, void* stream);
+
+/*
  * Append (page "mstar.engine.resources.attn.config", AttentionStep: a step's own tokens join
  * its KV stream; page "mstar.engine.resources.attn.cross": a stream is written through
  * ordinary Segments).  Writes the append_indptr[b+1] - append_indptr[b] new tokens of
@@ -294,9 +311,10 @@ int rae_read_kernel_timing(rae_ctx* ctx, float* attn_ms, float* merge_ms, int32_
  * num_merge_rows, batch, total_q, block_size, word offsets of the CTA pointer array and of
  * the tiles, the number of split units, word offsets of the four request arrays, the largest
  * rows per unit) followed by those arrays, packed; out->image_words words are used.
- * Tiles are 12 words {request, kv_head, first query token, query tokens, first key, end key,
- * first partial row or -1, split index, arrival counter of the split unit or -1, number of
- * splits of the unit, 0, 0}.
+ * Tiles are 12 words {request, first KV head, first query token, query tokens, first key,
+ * end key, first partial row or -1, split index, arrival counter of the split unit or -1,
+ * number of splits of the unit, KV heads of the unit, 0}.  A unit's rows are (token, query
+ * head) pairs, token-major, over the query heads of its KV heads.
  */
 int rae_plan_paged_host(const rae_config* cfg, const int32_t* qo_indptr,
                         const int32_t* kv_page_indptr, const int32_t* kv_page_indices,

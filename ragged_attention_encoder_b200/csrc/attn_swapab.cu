@@ -481,7 +481,8 @@ __global__ void __launch_bounds__(kSwThreads, 1) attn_swapab_kernel(const __grid
       if (tile.part >= 0 &&
           split_unit_complete(plan.counters, tile, &bar.merge_in, &bar.merge_out, &bar.merge_flag,
                               split_seen++, threadIdx.x == 0, lane, wc, &ok) && ok)
-        merge_split_unit<kD, 4>(tile, geo, p.part_o, p.part_lse, p.out, threadIdx.x, 128);
+        merge_split_unit<kD, 4>(tile, geo, tile.kv_head * geo.g, geo.g, p.part_o, p.part_lse, p.out,
+                                threadIdx.x, 128);
     }
   }
 

@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         if (tile.part >= 0 &&
             split_unit_complete(plan.counters, tile, &bar.merge_in, &bar.merge_out, &bar.merge_flag,
                                 split_seen++, false, lane, wc, &ok))
-          merge_split_unit<D, 8>(tile, geo, p.part_o, p.part_lse, p.out, threadIdx.x, 256);
+          merge_split_unit<D, 8>(tile, geo, tile.kv_head * geo.g, geo.g, p.part_o, p.part_lse, p.out, threadIdx.x, 256);
         continue;
       }
       const int tok = qt * tpt + tok_in_tile;     // token index within the work tile
@@ -553,7 +553,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       if (split &&
           split_unit_complete(plan.counters, tile, &bar.merge_in, &bar.merge_out, &bar.merge_flag,
                               split_seen++, threadIdx.x == 0, lane, wc, &ok))
-        merge_split_unit<D, 8>(tile, geo, p.part_o, p.part_lse, p.out, threadIdx.x, 256);
+        merge_split_unit<D, 8>(tile, geo, tile.kv_head * geo.g, geo.g, p.part_o, p.part_lse, p.out, threadIdx.x, 256);
     }
   }
 

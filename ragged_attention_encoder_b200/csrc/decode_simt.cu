@@ -4,18 +4,21 @@
 // of the decoder's packed queries over the context pages.  With one query token and a
 // handful of heads per KV head there are at most 8 query rows per (request, KV head), about
 // one multiply-add per byte of K/V read: HBM bound, far below the tensor-core ridge.  So this
-// kernel runs on CUDA cores and spends its effort on keeping HBM busy:
+// kernel runs on CUDA cores and spends its effort on keeping HBM busy with long reads:
 //
-//   * persistent CTAs walk the plan's tile list (balanced split-KV pieces);
-//   * a producer warp streams 16-key chunks of K and V pages with cp.async.bulk into a
-//     ring of shared-memory stages (4 chunks of K and 4 of V per stage, each chunk one
-//     contiguous 16 x d run of a page), signalled by mbarrier transaction counts;
-//   * four consumer warps each take one chunk per stage: scores with 16-byte vector reads,
-//     reduced over the lanes that share a key with warp shuffles; online softmax in fp32
-//     (scale folded into exp2); P.V accumulated in registers;
-//   * at the end of a tile the four warps' (max, sum, O) are merged through shared memory
-//     and the tile writes bf16 output, or an fp32 partial plus its log2-sum-exp when the
-//     plan split the unit's keys.
+//   * persistent CTAs walk the plan's tile list (balanced split-KV pieces); a work unit is
+//     (request, up to four adjacent KV heads, key range);
+//   * a producer warp streams 16-key chunks of K and V with cp.async.bulk into a ring of
+//     shared-memory stages.  A stage holds one chunk of every KV head of the unit.  With
+//     16-token pages the chunk is a whole page, and the unit's heads are adjacent in the pool
+//     [pages, Hkv, P, d], so each stage is ONE contiguous run of heads x 16 x d for K and one
+//     for V (8 KB each at d = 64 and four heads, instead of four 2 KB runs); stages are
+//     signalled by mbarrier transaction counts;
+//   * consumer warp w owns KV head w of the unit for the whole key range: scores with 16-byte
+//     vector reads, reduced over the lanes that share a key with warp shuffles; online
+//     softmax in fp32 (scale folded into exp2); P.V accumulated in registers.  A warp sees
+//     every key of its head, so no cross-warp merge is needed: each warp writes its rows as
+//     bf16, or as an fp32 partial plus its log2-sum-exp when the plan split the unit's keys.
 #include "kernels.h"
 #include "merge.cuh"
 #include "ptx.cuh"
@@ -30,7 +33,7 @@ __device__ int g_silent_producer_cta = -1;
 
 namespace {
 
-constexpr int kSimtConsumers = 4;
+constexpr int kSimtConsumers = kSimtMaxHeads;   // one consumer warp per KV head of a unit
 constexpr int kSimtThreads = (kSimtConsumers + 1) * 32;
 
 template <int D>
@@ -44,13 +47,10 @@ struct SimtCfg {
   static constexpr int STAGE_ELEMS = 2 * kSimtConsumers * CHUNK_ELEMS;   // K chunks, V chunks
 };
 
-template <int D, int R>
+template <int D>
 struct SimtSmem {
   using C = SimtCfg<D>;
-  __nv_bfloat16 stage[C::NST][C::STAGE_ELEMS];
-  float cm[kSimtConsumers][R];
-  float cl[kSimtConsumers][R];
-  float cacc[kSimtConsumers][R][D];
+  __nv_bfloat16 stage[C::NST][C::STAGE_ELEMS];   // [K: head][16][d], then [V: head][16][d]
   uint64_t full[C::NST];
   uint64_t empty[C::NST];
   uint64_t merge_in, merge_out;   // split-unit arrival protocol
@@ -59,14 +59,14 @@ struct SimtSmem {
 };
 
 template <int D, int R>
-__global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
+__global__ void __maxnreg__(200) decode_simt_kernel(
     DevPlan plan, Geometry geo, const __nv_bfloat16* __restrict__ q,
     const __nv_bfloat16* __restrict__ k_pool, const __nv_bfloat16* __restrict__ v_pool,
     __nv_bfloat16* __restrict__ out, float* __restrict__ part_o, float* __restrict__ part_lse,
     int* err, float scale_log2, int64_t timeout_ns) {
   using C = SimtCfg<D>;
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  auto& sm = *reinterpret_cast<SimtSmem<D, R>*>(smem_raw);
+  auto& sm = *reinterpret_cast<SimtSmem<D>*>(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -87,11 +87,14 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
 
   const int t_begin = plan.cta_ptr[blockIdx.x];
   const int t_end = plan.cta_ptr[blockIdx.x + 1];
+  const int P = geo.page_size;
 
   if (warp == kSimtConsumers) {
     // ------------------------------------------------------------- producer warp
-    // Lane i issues the copies of chunk i of a stage; each lane reads its chunk's page id
-    // before the stage's empty-barrier wait, so those reads overlap it and each other.
+    // The page ids of 32 chunks at a time are read one per lane (the reads overlap each
+    // other and the stage waits); lane 0 takes the waits and arms the transaction counts.
+    // With P == 16 a stage is two copies (K and V, all heads of the unit); otherwise lanes
+    // 0 .. nh-1 copy the heads' K chunks and lanes nh .. 2 nh - 1 their V chunks.
     const uint64_t pol = policy_evict_first();
     uint32_t use = 0;
     bool ok = true;
@@ -101,27 +104,36 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
     for (int t = t_begin; t < t_end && ok; ++t) {
       const Tile tile = plan.tiles[t];
       const int nch = (tile.kv1 - tile.kv0 + kSimtChunkKeys - 1) / kSimtChunkKeys;
+      const int nh = tile.nkvh;
       const int32_t* pages = plan.d + plan.c[tile.req];
-      for (int c0 = 0; c0 < nch; c0 += kSimtConsumers, ++use) {
-        const int s = use % C::NST;
-        const int cnt = min(kSimtConsumers, nch - c0);
-        int64_t row = 0;
-        if (lane < cnt) {
-          const int key = tile.kv0 + (c0 + lane) * kSimtChunkKeys;
-          const int page = pages[key / geo.page_size];
-          row = (int64_t(page) * geo.hkv + tile.kv_head) * geo.page_size + key % geo.page_size;
-        }
-        if (lane == 0 && use >= uint32_t(C::NST))
-          ok = wait_bounded(&sm.empty[s], ((use / C::NST) - 1) & 1, wc, 101);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], uint32_t(cnt) * 2u * C::CHUNK_BYTES);
-        __syncwarp();
-        if (lane < cnt) {
-          bulk_load(&sm.stage[s][lane * C::CHUNK_ELEMS], k_pool + row * D, C::CHUNK_BYTES,
-                    &sm.full[s], pol);
-          bulk_load(&sm.stage[s][(kSimtConsumers + lane) * C::CHUNK_ELEMS], v_pool + row * D,
-                    C::CHUNK_BYTES, &sm.full[s], pol);
+      for (int c0 = 0; c0 < nch && ok; c0 += 32) {
+        int my_page = 0;
+        if (c0 + lane < nch) my_page = pages[(tile.kv0 + (c0 + lane) * kSimtChunkKeys) / P];
+        const int cend = min(nch - c0, 32);
+        for (int ci = 0; ci < cend; ++ci, ++use) {
+          const int s = use % C::NST;
+          const int page = __shfl_sync(0xffffffffu, my_page, ci);
+          const int slot = (tile.kv0 + (c0 + ci) * kSimtChunkKeys) % P;
+          if (lane == 0 && use >= uint32_t(C::NST))
+            ok = wait_bounded(&sm.empty[s], ((use / C::NST) - 1) & 1, wc, 101);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], uint32_t(nh) * 2u * C::CHUNK_BYTES);
+          __syncwarp();
+          // first pool row of head tile.kv_head of this chunk
+          const int64_t row0 = (int64_t(page) * geo.hkv + tile.kv_head) * P + slot;
+          if (P == kSimtChunkKeys) {
+            if (lane < 2)
+              bulk_load(&sm.stage[s][lane * kSimtConsumers * C::CHUNK_ELEMS],
+                        (lane == 0 ? k_pool : v_pool) + row0 * D, uint32_t(nh) * C::CHUNK_BYTES,
+                        &sm.full[s], pol);
+          } else if (lane < 2 * nh) {
+            const int kv = lane >= nh;             // 0: K, 1: V
+            const int h = lane - kv * nh;
+            bulk_load(&sm.stage[s][(kv * kSimtConsumers + h) * C::CHUNK_ELEMS],
+                      (kv ? v_pool : k_pool) + (row0 + int64_t(h) * P) * D, C::CHUNK_BYTES,
+                      &sm.full[s], pol);
+          }
         }
       }
     }
@@ -145,15 +157,18 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
   uint32_t use = 0, split_seen = 0;
   for (int t = t_begin; t < t_end; ++t) {
     const Tile tile = plan.tiles[t];
-    const int rows = tile.qn * geo.g;
+    const bool active = warp < tile.nkvh;          // this warp's KV head is in the unit
+    const int kvh = tile.kv_head + warp;
+    const int rows = tile.qn * geo.g;              // rows of this warp's KV head
+    const int hpt = tile.nkvh * geo.g;             // query heads per token in the unit
     const int nch = (tile.kv1 - tile.kv0 + kSimtChunkKeys - 1) / kSimtChunkKeys;
 
     float qf[R][8];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      if (r < rows) {
+      if (active && r < rows) {
         const int tok = tile.q0 + r / geo.g;
-        const int head = tile.kv_head * geo.g + r % geo.g;
+        const int head = kvh * geo.g + r % geo.g;
         const uint4 v = *reinterpret_cast<const uint4*>(q + (int64_t(tok) * geo.hq + head) * D + cl * 8);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -188,15 +203,14 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
       for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
     }
 
-    for (int c0 = 0; c0 < nch; c0 += kSimtConsumers, ++use) {
+    for (int c = 0; c < nch; ++c, ++use) {
       const int s = use % C::NST;
       const bool ok = wait_bounded(&sm.full[s], (use / C::NST) & 1, wc, 102);
-      const int chunk = c0 + warp;
-      if (ok && chunk < nch) {
+      if (ok && active) {
         const uint4* kc = reinterpret_cast<const uint4*>(&sm.stage[s][warp * C::CHUNK_ELEMS]);
         const uint4* vc =
             reinterpret_cast<const uint4*>(&sm.stage[s][(kSimtConsumers + warp) * C::CHUNK_ELEMS]);
-        const int kbase = tile.kv0 + chunk * kSimtChunkKeys;
+        const int kbase = tile.kv0 + c * kSimtChunkKeys;
         float x[R][C::ITERS];
 #pragma unroll
         for (int i = 0; i < C::ITERS; ++i) {
@@ -275,44 +289,28 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
         for (int e = 0; e < 8; ++e) acc[r][e] += __shfl_xor_sync(0xffffffffu, acc[r][e], o);
       }
     }
-    if (grp == 0) {
-#pragma unroll
-      for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sm.cacc[warp][r][cl * 8 + e] = acc[r][e];
-    }
-    if (lane == 0) {
+    if (active && grp == 0 && !sm.abort) {
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        sm.cm[warp][r] = m[r];
-        sm.cl[warp][r] = l[r];
-      }
-    }
-    named_bar_sync(1, kSimtConsumers * 32);
-    if (!sm.abort) {
-      for (int e = threadIdx.x; e < rows * D; e += kSimtConsumers * 32) {
-        const int r = e / D;
-        const int dc = e - r * D;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kSimtConsumers; ++w) mx = fmaxf(mx, sm.cm[w][r]);
-        float num = 0.f, den = 0.f;
-        if (mx != -INFINITY) {
-#pragma unroll
-          for (int w = 0; w < kSimtConsumers; ++w) {
-            const float f = fast_exp2(sm.cm[w][r] - mx);
-            num += f * sm.cacc[w][r][dc];
-            den += f * sm.cl[w][r];
-          }
-        }
-        const float o = den > 0.f ? num / den : 0.f;
+        if (r >= rows) break;
+        const float inv = l[r] > 0.f ? 1.f / l[r] : 0.f;
+        const int tok = tile.q0 + r / geo.g;
+        const int gi = r % geo.g;
         if (tile.part < 0) {
-          const int tok = tile.q0 + r / geo.g;
-          const int head = tile.kv_head * geo.g + r % geo.g;
-          out[(int64_t(tok) * geo.hq + head) * D + dc] = __float2bfloat16_rn(o);
+          uint4 pk;
+          pk.x = pack_bf16x2(acc[r][0] * inv, acc[r][1] * inv);
+          pk.y = pack_bf16x2(acc[r][2] * inv, acc[r][3] * inv);
+          pk.z = pack_bf16x2(acc[r][4] * inv, acc[r][5] * inv);
+          pk.w = pack_bf16x2(acc[r][6] * inv, acc[r][7] * inv);
+          *reinterpret_cast<uint4*>(out + (int64_t(tok) * geo.hq + kvh * geo.g + gi) * D + cl * 8) = pk;
         } else {
-          part_o[int64_t(tile.part + r) * D + dc] = o;
-          if (dc == 0) part_lse[tile.part + r] = den > 0.f ? mx + fast_log2(den) : -INFINITY;
+          // unit row: (token, query head within the unit), token-major
+          const int urow = (r / geo.g) * hpt + warp * geo.g + gi;
+          float4* dst = reinterpret_cast<float4*>(part_o + int64_t(tile.part + urow) * D + cl * 8);
+          dst[0] = make_float4(acc[r][0] * inv, acc[r][1] * inv, acc[r][2] * inv, acc[r][3] * inv);
+          dst[1] = make_float4(acc[r][4] * inv, acc[r][5] * inv, acc[r][6] * inv, acc[r][7] * inv);
+          if (cl == 0)
+            part_lse[tile.part + urow] = l[r] > 0.f ? m[r] + fast_log2(l[r]) : -INFINITY;
         }
       }
     }
@@ -323,9 +321,9 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(
                                             &sm.merge_flag, split_seen++, threadIdx.x == 0, lane,
                                             wc, &ok);
       if (last && !sm.abort)
-        merge_split_unit<D, 32 / (D / 4)>(tile, geo, part_o, part_lse, out, threadIdx.x, kSimtConsumers * 32);
+        merge_split_unit<D, 32 / (D / 4)>(tile, geo, tile.kv_head * geo.g, hpt, part_o, part_lse,
+                                          out, threadIdx.x, kSimtConsumers * 32);
     }
-    named_bar_sync(1, kSimtConsumers * 32);
   }
 }
 
@@ -333,7 +331,7 @@ template <int D, int R>
 cudaError_t launch_t(const DevPlan& plan, const Geometry& geo, const void* q, const void* k_pool,
                      const void* v_pool, void* out, float* part_o, float* part_lse, int* err,
                      float scale_log2, int64_t timeout_ns, cudaStream_t stream) {
-  const size_t smem = sizeof(SimtSmem<D, R>);
+  const size_t smem = sizeof(SimtSmem<D>);
   auto kern = decode_simt_kernel<D, R>;
   static bool attr_set = false;   // per template instance; the attribute is per function
   if (!attr_set) {

@@ -52,15 +52,20 @@ __device__ __forceinline__ bool split_unit_complete(int* counters, const Tile& t
 // one coalesced read; each warp keeps kRows rows in flight (a multiple of the rows per warp
 // pass) and combines the splits in one online pass (running maximum, rescaled sums), in
 // split order.
+//
+// A unit's rows are (token, query head) pairs, token-major: row r is token tile.q0 + r / hpt,
+// query head head0 + r % hpt, where hpt is the number of query heads per token in the unit
+// (g for one KV head; g times the KV heads of the unit when it holds several).
 template <int D, int kRows>
-__device__ __forceinline__ void merge_split_unit(const Tile& tile, const Geometry& geo,
-                                                 const float* part_o, const float* part_lse,
-                                                 __nv_bfloat16* out, int tid, int nthreads) {
+__device__ __forceinline__ void merge_split_unit(const Tile& tile, const Geometry& geo, int head0,
+                                                 int hpt, const float* part_o,
+                                                 const float* part_lse, __nv_bfloat16* out,
+                                                 int tid, int nthreads) {
   constexpr int V = D / 4;              // float4 column groups per row
   constexpr int RPW = 32 / V;           // rows per warp and pass
   constexpr int U = kRows / RPW;        // passes unrolled
   static_assert(U >= 1 && U * RPW == kRows, "kRows must be a multiple of the rows per pass");
-  const int rows = tile.qn * geo.g;
+  const int rows = tile.qn * hpt;
   const int base = tile.part - tile.split * rows;
   const int ns = tile.nsplit;
   const int lane = tid & 31;
@@ -108,8 +113,8 @@ __device__ __forceinline__ void merge_split_unit(const Tile& tile, const Geometr
       const int r = r0 + u * RPW + rsub;
       if (r >= rows) continue;
       const float inv = den[u] > 0.f ? 1.f / den[u] : 0.f;
-      const int tok = tile.q0 + r / geo.g;
-      const int head = tile.kv_head * geo.g + r % geo.g;
+      const int tok = tile.q0 + r / hpt;
+      const int head = head0 + r % hpt;
       uint2 pk;
       pk.x = pack_bf16x2(acc[u].x * inv, acc[u].y * inv);
       pk.y = pack_bf16x2(acc[u].z * inv, acc[u].w * inv);

@@ -35,7 +35,7 @@ int32_t ceil_div32(int32_t a, int32_t b) {
 int64_t align4(int64_t w) { return (w + 3) & ~int64_t(3); }
 
 struct Unit {
-  int32_t req, kvh, q0, qn, nkeys, rows;
+  int32_t req, kvh, nkvh, q0, qn, nkeys, rows;
   int32_t w;       // cost of one key block (the scheduler's unit; see tc_block_cost)
   int64_t group;   // units of one group read the same K/V (one request or span, one KV head)
 };
@@ -349,7 +349,7 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
                  : int32_t(part_base[size_t(p.unit)] + int64_t(t.split) * un.rows);
     t.munit = int32_t(munit[size_t(p.unit)]);
     t.nsplit = npieces[size_t(p.unit)];
-    t.pad0 = 0;
+    t.nkvh = un.nkvh;
     t.pad1 = 0;
     sc->tiles[i] = t;
   }
@@ -453,21 +453,27 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
   const int32_t tok_per_unit =
       simt ? std::max(max_qlen, 1) : (swap ? swap_n / g : 2 * tile_tok);
 
+  // A decode unit holds up to kSimtMaxHeads adjacent KV heads (one per consumer warp), so
+  // that each 16-key chunk of a page is read as one run over those heads; the other kernels
+  // take one KV head per unit.
+  const int32_t hpu = simt ? kSimtMaxHeads : 1;
   std::vector<Unit> units;
   for (int32_t b = 0; b < batch; ++b) {
     const int32_t qlen = qo_indptr[b + 1] - qo_indptr[b];
-    for (int32_t h = 0; h < cfg.num_kv_heads; ++h)
+    for (int32_t h = 0; h < cfg.num_kv_heads; h += hpu)
       for (int32_t t = 0; t < qlen; t += tok_per_unit) {
         Unit u;
         u.req = b;
         u.kvh = h;
+        u.nkvh = std::min(hpu, cfg.num_kv_heads - h);
         u.q0 = qo_indptr[b] + t;
         u.qn = std::min(tok_per_unit, qlen - t);
         // causal: the unit's last query (local index t + qn - 1) sees kv_len - qlen + t + qn
         // keys; no row of the unit sees more
         u.nkeys = causal ? kv_len[b] - qlen + t + u.qn : kv_len[b];
-        u.rows = u.qn * g;
-        u.w = (simt || swap) ? 1 : tc_block_cost(ceil_div32(u.qn, tile_tok));
+        u.rows = u.qn * g * u.nkvh;
+        // decode: a block's bytes grow with the unit's heads
+        u.w = simt ? u.nkvh : swap ? 1 : tc_block_cost(ceil_div32(u.qn, tile_tok));
         u.group = int64_t(b) * cfg.num_kv_heads + h;
         units.push_back(u);
       }
@@ -477,8 +483,9 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
   out->total_q = total_q;
   out->block_size = causal ? 1 : 0;
   out->kv_extent = page_extent;
+  // rows per unit and KV head: what the kernel is instantiated for
   int32_t rows_max = 0;
-  for (const Unit& u : units) rows_max = std::max(rows_max, u.rows);
+  for (const Unit& u : units) rows_max = std::max(rows_max, u.rows / u.nkvh);
   if (swap) rows_max = swap_n;   // the row count the swapped kernel is instantiated for
   out->rows_max = rows_max;
   Schedule sc;
@@ -526,6 +533,7 @@ int build_ragged_plan(const rae_config& cfg, const int32_t* cu_q, const int32_t*
         Unit u;
         u.req = s;
         u.kvh = h;
+        u.nkvh = 1;
         u.q0 = cu_q[s] + t;
         u.qn = std::min(tok_per_unit, lq - t);
         int64_t lim = lk;

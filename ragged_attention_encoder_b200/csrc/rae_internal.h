@@ -49,7 +49,8 @@ struct Tile {
   int32_t split;      // split index within the unit (0 when unsplit)
   int32_t munit;      // split unit (index of its arrival counter); -1 when unsplit
   int32_t nsplit;     // splits of the unit (1 when unsplit)
-  int32_t pad0, pad1;
+  int32_t nkvh;       // KV heads of the unit: kv_head ... kv_head + nkvh - 1 (1 except decode)
+  int32_t pad1;
 };
 static_assert(sizeof(Tile) == 48, "tile is 12 words");
 
@@ -58,6 +59,10 @@ static_assert(sizeof(Tile) == 48, "tile is 12 words");
 constexpr int32_t kTcBlockKeys = 128;
 constexpr int32_t kSimtChunkKeys = 16;
 constexpr int32_t kSimtMaxRows = 8;
+// Most KV heads in a decode unit: one per consumer warp of the decode kernel, so that a
+// 16-key chunk of a page is one contiguous run of the unit's heads (pool layout
+// [pages, Hkv, P, d]).  A request's KV heads form units of this many, the last one fewer.
+constexpr int32_t kSimtMaxHeads = 4;
 constexpr int32_t kTcRows = 128;
 
 // Workspace layout: [error words | slot 0 image | slot 1 image | write staging | partial O |

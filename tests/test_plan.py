@@ -43,12 +43,16 @@ def test_test_build_exports_its_hooks_and_the_product_does_not(built_library):
 
 
 def _tiles_rows(tiles, g):
-    """Expand tiles into (token, head, kv0, kv1, tile index)."""
+    """Expand tiles into (token, head, kv0, kv1, tile index).  A tile's unit holds the KV
+    heads kvh ... kvh + nkvh - 1 (word 10); its rows are (token, query head), token-major."""
     out = []
     for i, t in enumerate(tiles):
         req, kvh, q0, qn, kv0, kv1, part, split = (int(x) for x in t[:8])
-        for r in range(qn * g):
-            out.append((q0 + r // g, kvh * g + r % g, kv0, kv1, i))
+        nkvh = int(t[10])
+        assert nkvh >= 1
+        hpt = g * nkvh
+        for r in range(qn * hpt):
+            out.append((q0 + r // hpt, kvh * g + r % hpt, kv0, kv1, i))
     return out
 
 
@@ -67,8 +71,9 @@ def _check_merge(p, g, hq):
     tiles = p["tiles"]
     units = {}
     for t in tiles:
-        req, kvh, q0, qn, kv0, kv1, part, split, munit, nsplit = (int(x) for x in t[:10])
-        units.setdefault((req, kvh, q0), []).append((split, kv0, kv1, part, qn, munit, nsplit))
+        req, kvh, q0, qn, kv0, kv1, part, split, munit, nsplit, nkvh = (int(x) for x in t[:11])
+        units.setdefault((req, kvh, q0), []).append((split, kv0, kv1, part, qn * nkvh, munit,
+                                                     nsplit))
     merge_rows = 0
     seen_parts, seen_units = set(), set()
     for key, pieces in units.items():
@@ -239,11 +244,12 @@ def test_empty_inputs_plan_nothing():
     assert p["raw"].num_tiles == 0
     p = plan_ragged_host([0, 0], None, 4, num_qo_heads=2, num_kv_heads=2, head_dim=64)
     assert p["raw"].num_tiles == 0
-    # a request with queries but no context keys gets one empty tile (it writes zeros)
+    # a request with queries but no context keys gets one empty tile per unit (it writes
+    # zeros); a decode unit holds both KV heads
     p = plan_paged_host([0, 2], [0, 0], [], [0], 1, num_qo_heads=4, num_kv_heads=2, head_dim=64,
                         page_size=16)
     t = p["tiles"]
-    assert t.shape[0] == 2 and np.all(t[:, 4] == 0) and np.all(t[:, 5] == 0)
+    assert t.shape[0] == 1 and t[0, 10] == 2 and t[0, 4] == 0 and t[0, 5] == 0
 
 
 @pytest.mark.parametrize("seed", range(6))
