@@ -58,6 +58,14 @@ def parse():
                     help="run only this workload's layer call --reps times (for ncu captures); "
                          "6: paged causal chunked prefill, 7: the fused K/V projection")
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--tp", action="store_true",
+                    help="tensor-parallel: the decode step's heads sharded over the --gpus ranks, "
+                         "each layer's o_proj partial summed by one all-reduce (strong scaling)")
+    ap.add_argument("--counters", action="store_true",
+                    help="capture the ncu counters of every workload's kernel (one launch each, "
+                         "a few metrics) and write them to --counters-out; prints no benchmark line")
+    ap.add_argument("--counters-out", default=None,
+                    help="file the counters go to (default profiles/counters.json)")
     return ap.parse_args()
 
 
@@ -127,27 +135,62 @@ def load_peaks():
                 "tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def load_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the kernel source."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+# Kernel of each workload's layer call, and the sources it is built from.
+PROFILE_CASES = {
+    1: ("tiny_paged_decode", "decode_simt_kernel", "decode_simt.cu"),
+    2: ("whisper_large_decode", "decode_simt_kernel", "decode_simt.cu"),
+    3: ("packed_multitoken_cross", "attn_tc_kernel", "attn_tc.cu"),
+    4: ("ragged_block_causal", "attn_tc_kernel", "attn_tc.cu"),
+    5: ("long_context_splitkv", "attn_swapab_kernel", "attn_swapab.cu"),
+    6: ("paged_causal_chunked_prefill", "attn_tc_kernel", "attn_tc.cu"),
+    7: ("whisper_encode_kv_projection_write", "project_write_kernel", "project_write.cu"),
+}
+COUNTER_METRICS = ("gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum,"
+                   "sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_elapsed,"
+                   "gpu__dram_throughput.avg.pct_of_peak_sustained_elapsed")
+COUNTERS_PATH = os.path.join(ROOT, "profiles", "counters.json")
+
+
+def kernel_source_sha(source: str) -> str:
+    """Hash of a kernel's .cu file and every header of the library's sources: counters are
+    only reported for the source they were taken on."""
+    import glob
+    import hashlib
+    csrc = os.path.join(ROOT, "ragged_attention_encoder_b200", "csrc")
+    h = hashlib.sha256()
+    files = [os.path.join(csrc, source)] + sorted(
+        glob.glob(os.path.join(csrc, "*.cuh")) + glob.glob(os.path.join(csrc, "*.h")))
+    for f in files:
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_counters(workload: str):
+    """The ncu counters of the workload's kernel from profiles/counters.json, if they were
+    taken on the current source (else None)."""
     try:
-        with open(path) as f:
+        with open(COUNTERS_PATH) as f:
             entries = json.load(f)
     except Exception:
         return None
-    import hashlib
     for e in entries:
-        if e.get("kernel") != kernel or e.get("workload") != workload:
+        if e.get("workload") != workload:
             continue
-        src = os.path.join(ROOT, e["source"])
         try:
-            with open(src, "rb") as f:
-                sha = hashlib.sha256(f.read()).hexdigest()[:16]
+            if kernel_source_sha(e["source"]) != e.get("source_sha"):
+                return None
         except Exception:
             return None
-        if sha == e.get("source_sha"):
-            return float(e["dram_bytes_per_launch"])
+        return e
     return None
+
+
+def load_traffic(workload: str):
+    """DRAM bytes (read + write) per launch of the workload's kernel, from the counters."""
+    e = load_counters(workload)
+    return None if e is None else float(e["dram_bytes_read"] + e["dram_bytes_write"])
 
 
 class ClockSampler:
@@ -337,6 +380,67 @@ def projection_row(dev, peaks, flush_buf):
     }
 
 
+def q_projection_row(i, dev, flush_buf):
+    """The Q projection in front of a layer call (page "mstar.model.components.attention",
+    CrossAttention: q = h . W_q^T + b_q, projected every step; hidden = Hq * d, seeded
+    synthetic weights): the cuBLAS GEMM and the run in sequence, against the run alone, with
+    what fusing the GEMM into the run's Q load could save at most (the q tensor's write and
+    read at the measured HBM peak, plus one launch).  Median of 30 calls, L2 flushed."""
+    import torch
+    import torch.nn.functional as F
+    case, ctx, plan, call, _, _, _ = setup_workload(i, dev)
+    tokens = int(case.qo_indptr[-1])
+    hidden = case.num_qo_heads * case.head_dim
+    gen = torch.Generator(device=dev).manual_seed(90 + i)
+    h = torch.randn(tokens, hidden, generator=gen, device=dev).to(torch.bfloat16)
+    w_q = (torch.randn(hidden, hidden, generator=gen, device=dev) / hidden ** 0.5).to(torch.bfloat16)
+    b_q = torch.randn(hidden, generator=gen, device=dev).to(torch.bfloat16)
+    q = case.q.to(dev)
+
+    def gemm():
+        q.copy_(F.linear(h, w_q, b_q).view_as(q))
+
+    def timed(fn):
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for _ in range(30):
+            flush_l2(flush_buf)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        return statistics.median(ts)
+
+    t_run = timed(call)
+    t_gemm = timed(lambda: F.linear(h, w_q, b_q))
+    t_both = timed(lambda: (gemm(), call()))
+    ctx.check_device_status()
+    q_bytes = tokens * hidden * 2
+    del ctx
+    return {"tokens": tokens, "hidden": hidden, "run_us": round(t_run, 2),
+            "q_gemm_us": round(t_gemm, 2), "gemm_then_run_us": round(t_both, 2),
+            "fusion_saves_at_most_us": round(2 * q_bytes / (6550.0 * 1e9) * 1e6 + 2.0, 2),
+            "note": "the bound counts q written and read once at 6550 GB/s plus 2 us of launch"}
+
+
+def counters_row(workload: str, algorithmic_bytes: int):
+    """ncu counters of the row's kernel (one launch, cold L2) taken on the current source, or
+    None: DRAM traffic per launch against the algorithmic bytes, tensor-pipe and DRAM
+    utilisation."""
+    e = load_counters(workload)
+    if e is None:
+        return None
+    traffic = e["dram_bytes_read"] + e["dram_bytes_write"]
+    return {"kernel": e["kernel"], "traffic": traffic,
+            "traffic_over_algorithmic": round(traffic / algorithmic_bytes, 3),
+            "tensor_pipe_pct": e["tensor_pipe_pct"], "dram_throughput_pct": e["dram_throughput_pct"],
+            "ncu_time_us": e["gpu_time_us"], "source_sha": e["source_sha"]}
+
+
 def workload_table(dev, peaks, flush_buf):
     """Per-layer-call numbers of the five workloads, and of paged causal chunked prefill (6):
     median of 100 calls after 10 warm-up calls, L2 flushed (a 256 MB write, over twice the
@@ -374,10 +478,18 @@ def workload_table(dev, peaks, flush_buf):
             "ctas": plan.num_ctas,
             "merge_rows": plan.num_merge_rows,
             "plan_host_us": round(plan_us, 1),
+            "counters": counters_row(case.name, nbytes),
         }
         del ctx
         torch.cuda.empty_cache()
+    rows["q_projection_then_run"] = {
+        "whisper_large_decode": q_projection_row(2, dev, flush_buf),
+        "packed_multitoken_cross": q_projection_row(3, dev, flush_buf)}
+    torch.cuda.empty_cache()
     rows["whisper_encode_kv_projection_write"] = projection_row(dev, peaks, flush_buf)
+    rows["whisper_encode_kv_projection_write"]["counters"] = counters_row(
+        "whisper_encode_kv_projection_write",
+        rows["whisper_encode_kv_projection_write"]["algorithmic_bytes"])
     torch.cuda.empty_cache()
     return rows
 
@@ -589,7 +701,7 @@ def run_ours(args):
     attn_mean_ms = statistics.fmean(attn_ms) if attn_ms else float("nan")
     launch_bytes = nbytes                        # one layer call's algorithmic bytes
     achieved = launch_bytes / (attn_mean_ms * 1e-3) / 1e9
-    traffic = load_traffic("decode_simt_kernel", "whisper_large_decode")
+    traffic = load_traffic("whisper_large_decode")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": traffic, "kernel": "decode_simt_kernel<64,1>",
@@ -641,6 +753,104 @@ def run_ours(args):
     if world == 1 and not args.skip_workloads:
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         result["workloads"] = workload_table(dev, peaks, flush)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------- tensor-parallel arm
+
+def run_tp(args):
+    """The Whisper-large decode step with its 20 heads sharded over the ranks (page
+    "mstar.model.components.distributed.attention", ParallelAttention): every rank plans and
+    runs its heads of each of the 32 layers, multiplies its attention output by its columns of
+    W_o (hidden 1280, synthetic seeded weights; rank 0 adds the bias) and takes part in one fp32
+    all-reduce per layer.  Total work is fixed as N grows (strong scaling); value counts the
+    unsharded layer's KV bytes per step over the slowest rank's device time."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    from ragged_attention_encoder_b200 import inputs
+    from ragged_attention_encoder_b200.tp import TensorParallelCrossAttention
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    case = inputs.workload(2)
+    hidden = case.num_qo_heads * case.head_dim          # Whisper-large: 1280
+    tp = TensorParallelCrossAttention(case.num_qo_heads, case.num_kv_heads, case.head_dim,
+                                      case.page_size, rank=rank, world=world, device=dev)
+    s = tp.shard
+    gen = torch.Generator(device=dev).manual_seed(2000 + rank)
+    shape = (case.num_pages, s.num_kv_heads, case.page_size, case.head_dim)
+    k_pools, v_pools, qs, ws, outs, projs = [], [], [], [], [], []
+    for _ in range(LAYERS):
+        k_pools.append(torch.randn(shape, generator=gen, device=dev, dtype=torch.bfloat16))
+        v_pools.append(torch.randn(shape, generator=gen, device=dev, dtype=torch.bfloat16))
+        qs.append(torch.randn((case.q.shape[0], s.num_qo_heads, case.head_dim), generator=gen,
+                              device=dev, dtype=torch.bfloat16))
+        ws.append((torch.randn((hidden, s.num_qo_heads * case.head_dim), generator=gen, device=dev)
+                   / hidden ** 0.5).to(torch.bfloat16))
+        outs.append(torch.empty_like(qs[-1]))
+        projs.append(torch.empty((case.q.shape[0], hidden), dtype=torch.float32, device=dev))
+    b_o = torch.randn(hidden, generator=gen, device=dev).to(torch.bfloat16)
+
+    def step():
+        plan = tp.plan(case.qo_indptr, case.kv_page_indptr, case.kv_page_indices, case.kv_len,
+                       case.num_pages)
+        for layer in range(LAYERS):
+            tp.forward(plan, qs[layer], k_pools[layer], v_pools[layer], ws[layer], b_o,
+                       outs[layer], projs[layer])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    tp.ctx.check_device_status()
+    sampler = ClockSampler(local)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    tp.ctx.check_device_status()
+    ms = max_over_ranks(t0.elapsed_time(t1), dev) / args.steps
+    flops, nbytes, _ = paged_work(case)
+    tokens = int(case.qo_indptr[-1])
+    proj_flops = 2 * tokens * hidden * hidden
+    value = nbytes * LAYERS / (ms * 1e-3) / 1e9
+    result = {
+        "metric": "KV HBM GB/s (Whisper-large decode cross-attention step with o_proj, heads "
+                  "sharded over the GPUs)",
+        "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (device-seeded pools, queries and W_o)",
+        "config": {"workload": "whisper_large_decode_tp", "requests": 64, "context_tokens": 1500,
+                   "num_qo_heads": 20, "num_kv_heads": 20, "head_dim": 64, "page_size": 16,
+                   "hidden": hidden, "layers_per_step": LAYERS,
+                   "heads_per_rank": s.num_qo_heads, "parallelism": f"tp{world}",
+                   "collective": "one fp32 all-reduce of [64, 1280] per layer (NCCL)"},
+        "us_per_layer_call": round(ms * 1e3 / LAYERS, 2),
+        "o_proj_tflop_per_step": round(proj_flops * LAYERS / 1e12, 4),
+        "gpu_launches": 2 * LAYERS * args.steps,
+        "clocks": clocks,
+        "e2e": None,
+    }
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -719,14 +929,78 @@ def run_profile_case(args):
     print(json.dumps({**info, "reps": args.reps}), flush=True)
 
 
+def _ncu_csv_metrics(path: str):
+    """{metric: value} of the single launch in an ncu --csv log (units as ncu prints them)."""
+    import csv
+    with open(path) as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    out = {}
+    for row in csv.DictReader(lines):
+        name, unit, val = row.get("Metric Name"), row.get("Metric Unit", ""), row.get("Metric Value")
+        if not name or val is None:
+            continue
+        v = float(val.replace(",", ""))
+        scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "nsecond": 1e-3,
+                 "ns": 1e-3, "usecond": 1.0, "us": 1.0, "msecond": 1e3, "ms": 1e3,
+                 "%": 1.0}.get(unit, 1.0)
+        out[name] = v * scale
+    return out
+
+
+def run_counters(args):
+    """ncu counters of every workload's kernel: each `--profile-case I` command runs once
+    plainly, then under ncu with a handful of metrics on one launch (the second of its
+    kernel; `--clock-control none`).  Writes profiles/counters.json."""
+    ncu = os.environ.get("NCU", "ncu")
+    outdir = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) \
+        else tempfile.mkdtemp()
+    entries = []
+    for case_id, (workload, kernel, source) in PROFILE_CASES.items():
+        cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--profile-case", str(case_id),
+               "--reps", "3"]
+        plain = subprocess.run(cmd, capture_output=True, text=True, timeout=600)
+        if plain.returncode != 0:
+            raise RuntimeError(f"profile case {case_id} failed without ncu:\n{plain.stderr[-2000:]}")
+        log = os.path.join(outdir, f"counters_{workload}.csv")
+        ncmd = [ncu, "--metrics", COUNTER_METRICS, "--clock-control", "none", "-k",
+                f"regex:{kernel}", "-s", "1", "-c", "1", "--csv", "--log-file", log] + cmd
+        t0 = time.time()
+        res = subprocess.run(ncmd, capture_output=True, text=True, timeout=900)
+        if res.returncode != 0:
+            raise RuntimeError(f"ncu on case {case_id} failed:\n{res.stdout[-2000:]}\n{res.stderr[-2000:]}")
+        m = _ncu_csv_metrics(log)
+        entries.append({
+            "workload": workload, "kernel": kernel, "source": source,
+            "source_sha": kernel_source_sha(source),
+            "gpu_time_us": round(m["gpu__time_duration.sum"], 2),
+            "dram_bytes_read": int(m["dram__bytes_read.sum"]),
+            "dram_bytes_write": int(m["dram__bytes_write.sum"]),
+            "tensor_pipe_pct": round(m["sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_elapsed"], 2),
+            "dram_throughput_pct": round(m["gpu__dram_throughput.avg.pct_of_peak_sustained_elapsed"], 2),
+            "command": " ".join(["ncu", "--metrics", COUNTER_METRICS, "--clock-control", "none",
+                                 "-k", f"regex:{kernel}", "-s", "1", "-c", "1", "python", "bench.py",
+                                 "--profile-case", str(case_id), "--reps", "3"]),
+            "capture_s": round(time.time() - t0, 1),
+        })
+        print(json.dumps(entries[-1]), flush=True)
+    with open(args.counters_out or COUNTERS_PATH, "w") as f:
+        json.dump(entries, f, indent=1)
+        f.write("\n")
+
+
 def main():
     args = parse()
+    if args.counters:
+        run_counters(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.profile_case is not None:
         run_profile_case(args)
     elif args.impl == "reference":
         run_reference(args)
+    elif args.tp:
+        run_tp(args)
     else:
         run_ours(args)
 

@@ -100,6 +100,29 @@ def test_long_context_splitkv_sampled():
                 assert_close(o[t, heads], ref, what=f"req {b} tok {t}")
 
 
+@pytest.mark.slow
+def test_long_context_splitkv_full():
+    """The whole long-context workload (8 requests x 4 tokens x 64 heads over 32k-131k keys),
+    compared element by element: every (request, KV head) with the float64 oracle's attention
+    over the request's context rows (the context write that placed them is bit-exact)."""
+    case = inputs.workload(5)
+    out, plan, *_ = run_paged(case)
+    assert plan.num_merge_rows > 0
+    g = case.num_qo_heads // case.num_kv_heads
+    ref = np.zeros(tuple(case.q.shape), dtype=np.float64)
+    scale = 1.0 / np.sqrt(case.head_dim)
+    for b in range(case.batch):
+        c0, c1 = int(case.cu_enc[b]), int(case.cu_enc[b + 1])
+        t0, t1 = int(case.qo_indptr[b]), int(case.qo_indptr[b + 1])
+        for kvh in range(case.num_kv_heads):
+            kb = oracle.as_f64(case.k_ctx[c0:c1, kvh])
+            vb = oracle.as_f64(case.v_ctx[c0:c1, kvh])
+            for h in range(kvh * g, kvh * g + g):
+                ref[t0:t1, h] = oracle.attention_rows(oracle.as_f64(case.q[t0:t1, h]), kb, vb,
+                                                      scale)
+    assert_close(out, ref, what="workload 5 (full)")
+
+
 # ---------------------------------------------------------------------------- edge cases
 
 @pytest.mark.parametrize("P", [16, 32, 64])

@@ -47,6 +47,17 @@ def test_ragged_block_causal_workload_sampled():
     assert_close(got, ref, what="workload 4")
 
 
+@pytest.mark.slow
+def test_ragged_block_causal_workload_full():
+    """The whole packed encoder workload (31 spans, 65 959 tokens, 16 heads, block 256) in the
+    benchmark's launch configuration, compared element by element with the float64 oracle
+    (about a minute of host time)."""
+    case = inputs.workload(4)
+    out, plan, *_ = run_ragged(case)
+    assert plan.num_ctas == 148
+    assert_close(out, oracle_ragged(case), what="workload 4 (full)")
+
+
 def test_two_span_cross_tiny():
     case = inputs.ragged_case(120, span_lens=[3, 1, 9, 0, 130, 5, 2, 40],
                               kv_span_lens=[30, 2, 17, 5, 1, 0, 300, 129], num_qo_heads=8,
