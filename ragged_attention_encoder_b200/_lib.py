@@ -85,6 +85,7 @@ SIGNATURES = {
     "rae_plan_paged_causal": (ctypes.c_int, [vp, i32, P32, P32, P32, P32, i32, i32, vp, vp,
                                              ctypes.POINTER(RaePlan)]),
     "rae_append_kv": (ctypes.c_int, [vp, vp, vp, P32, P32, P32, P32, i32, vp, vp, i32, vp, vp]),
+    "rae_o_proj_partial": (ctypes.c_int, [vp, vp, i32, i32, vp, i32, vp, vp, vp, vp]),
     "rae_project_write_context": (ctypes.c_int, [vp, vp, i32, vp, vp, vp, vp, P32, P32, P32, i32,
                                                  vp, vp, i32, vp, vp]),
     "rae_run_paged": (ctypes.c_int, [vp, ctypes.POINTER(RaePlan), vp, vp, vp, i32, vp,

@@ -236,6 +236,31 @@ class Context:
             _ptr32(ix) if ix.size else None, batch, _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
             int(k_pool.shape[0]), self.workspace.data_ptr(), _stream_handle(self.device)))
 
+    def o_proj_partial(self, attn, w_o, bias=None, out=None):
+        """One tensor-parallel rank's output projection: attn [m, Hq, d] (this context's heads,
+        the run's output) or [m, Hq * d], times w_o [n, Hq * d] (the rank's columns of W_o,
+        nn.Linear layout), plus bias [n] (bf16, or None); returns out [m, n] fp32.  The ranks'
+        outputs sum to the full projection."""
+        import torch
+        m = int(attn.shape[0])
+        k = self.num_qo_heads * self.head_dim
+        if attn.numel() != m * k or attn.dtype != torch.bfloat16 or not attn.is_contiguous():
+            raise ValueError("attn must be a contiguous bf16 [m, num_qo_heads, head_dim] tensor")
+        if w_o.dim() != 2 or w_o.shape[1] != k or w_o.dtype != torch.bfloat16:
+            raise ValueError("w_o must be bf16 [n, num_qo_heads * head_dim]")
+        n = int(w_o.shape[0])
+        if bias is not None and (tuple(bias.shape) != (n,) or bias.dtype != torch.bfloat16):
+            raise ValueError("bias must be bf16 [n]")
+        if out is None:
+            out = torch.empty((m, n), dtype=torch.float32, device=self.device)
+        elif tuple(out.shape) != (m, n) or out.dtype != torch.float32 or not out.is_contiguous():
+            raise ValueError("out must be a contiguous fp32 [m, n] tensor")
+        self._check(self._lib.rae_o_proj_partial(
+            self._h, _dev(attn, "attn"), m, k, _dev(w_o, "w_o"), n,
+            None if bias is None else _dev(bias, "bias"), _dev(out, "out", torch.float32),
+            self.workspace.data_ptr(), _stream_handle(self.device)))
+        return out
+
     def append_kv(self, k_new, v_new, append_indptr, kv_page_indptr, kv_page_indices, kv_len,
                   k_pool, v_pool):
         """Writes each request's new tokens (rows append_indptr[b]... of k_new / v_new) to the

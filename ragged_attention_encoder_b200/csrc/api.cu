@@ -405,6 +405,44 @@ int rae_project_write_context(rae_ctx* ctx, const void* hidden, int32_t hidden_d
   return RAE_OK;
 }
 
+int rae_o_proj_partial(rae_ctx* ctx, const void* attn, int32_t m, int32_t k, const void* w_o,
+                       int32_t n, const void* bias, void* out, void* workspace, void* stream) {
+  if (!ctx) return RAE_ERR_INVALID_ARG;
+  if (m < 0 || k <= 0 || n <= 0) return set_err(ctx, RAE_ERR_INVALID_ARG, "bad o_proj sizes");
+  if (k % 64 != 0 || n % o_proj_tile_cols() != 0)
+    return set_err(ctx, RAE_ERR_UNSUPPORTED, "o_proj needs k % 64 == 0 and n % 128 == 0");
+  if (m > int64_t(65535) * 128) return set_err(ctx, RAE_ERR_CAPACITY, "more than 8388480 rows");
+  if (m == 0) return RAE_OK;
+  if (!attn || !w_o || !out || !workspace)
+    return set_err(ctx, RAE_ERR_INVALID_ARG, "NULL device pointer");
+  if (!aligned16(attn) || !aligned16(w_o) || !aligned16(bias) || !aligned16(out))
+    return set_err(ctx, RAE_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
+  OProjArgs a;
+  int rc;
+  {
+    const cuuint64_t dims[2] = {cuuint64_t(k), cuuint64_t(m)};
+    const cuuint64_t strides[1] = {cuuint64_t(k) * 2};
+    const cuuint32_t box[2] = {64, 128};
+    if ((rc = make_map(ctx, &a.maps[0], attn, 2, dims, strides, box))) return rc;
+  }
+  {
+    const cuuint64_t dims[2] = {cuuint64_t(k), cuuint64_t(n)};
+    const cuuint64_t strides[1] = {cuuint64_t(k) * 2};
+    const cuuint32_t box[2] = {64, cuuint32_t(o_proj_tile_cols())};
+    if ((rc = make_map(ctx, &a.maps[1], w_o, 2, dims, strides, box))) return rc;
+  }
+  a.bias = bias;
+  a.out = out;
+  a.err = reinterpret_cast<int*>(workspace);
+  a.timeout_ns = ctx->timeout_ns;
+  a.m = m;
+  a.n = n;
+  a.k = k;
+  cudaError_t e = launch_o_proj(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_err(ctx, e, "o_proj kernel launch");
+  return RAE_OK;
+}
+
 int rae_append_kv(rae_ctx* ctx, const void* k_new, const void* v_new,
                   const int32_t* append_indptr, const int32_t* kv_page_indptr,
                   const int32_t* kv_page_indices, const int32_t* kv_len, int32_t batch,

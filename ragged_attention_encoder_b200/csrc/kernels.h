@@ -91,6 +91,19 @@ struct ProjectWriteArgs {
 };
 cudaError_t launch_project_write(const ProjectWriteArgs& args, cudaStream_t stream);
 
+// One tensor-parallel rank's o_proj partial: out [m, n] fp32 = attn [m, k] . w [n, k]^T
+// (+ bias [n]); n % 128 == 0, k % 64 == 0.
+struct OProjArgs {
+  CUtensorMap maps[2];       // attn {k, m} box {64, 128}; w {k, n} box {64, 128}
+  const void* bias;          // [n] bf16 or null
+  void* out;                 // [m, n] fp32
+  int* err;
+  int64_t timeout_ns;
+  int32_t m, n, k;
+};
+cudaError_t launch_o_proj(const OProjArgs& args, cudaStream_t stream);
+int o_proj_tile_cols();
+
 // Message of the calling thread's last failing context-free call (rae_write_context_noalloc).
 const char* noalloc_last_error();
 // Output columns per tile of the projection kernel (the weight maps' box height).
