@@ -45,6 +45,7 @@ struct Unit {
 // takes about as long with one 128-row query tile as with two (measured 1.05x for two full
 // tiles against one), so a unit's cost follows its key blocks, not its rows.
 constexpr int32_t kTcStep = 16;
+constexpr int32_t kTcLptSlackPct = 15;
 int32_t tc_block_cost(int32_t tiles) { return tiles > 1 ? kTcStep + 1 : kTcStep; }
 
 struct Piece {
@@ -138,9 +139,12 @@ int emit_image(const Schedule& sc, const int32_t* a, int64_t na, const int32_t* 
 //   blk: keys per block; ovh: per-tile overhead in the units of Unit::w; g: query heads per
 //   KV head.
 //   lpt_factor: whole units are scheduled longest-first when every CTA's share is at least
-//   lpt_factor times the largest unit; otherwise the balanced contiguous partition is used.
+//   lpt_factor times the largest unit; otherwise the balanced contiguous partition is used,
+//   unless whole units (longest-first) leave the busiest CTA within lpt_slack_pct per cent of
+//   the partition's (0: never).
 int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units, int32_t blk,
-             int32_t ovh, int32_t g, int32_t lpt_factor, Schedule* sc, std::string* err) {
+             int32_t ovh, int32_t g, int32_t lpt_factor, int32_t lpt_slack_pct, Schedule* sc,
+             std::string* err) {
   const int32_t grid = grid_for(cfg, kind);
   const int64_t nu = int64_t(units.size());
   std::vector<int64_t> nb(nu), cost(nu);
@@ -158,39 +162,38 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
 
   auto lpt = [&]() {
     // Whole units, each to the least-loaded CTA, in an order that keeps the units sharing
-    // K/V together in time (so their K/V stay in L2) and still starts the big work first:
-    // groups by descending total cost, units within a group by descending cost.
+    // K/V together in time and still starts the big work first: groups by descending largest
+    // unit, units within a group by descending cost.  Consecutive units go to different CTAs
+    // that are free at about the same time, so the units of a group (its query chunks) run
+    // side by side and read their common K/V blocks through L2 once.
     pieces.clear();
     std::fill(npieces.begin(), npieces.end(), 0);
-    std::vector<int64_t> order(nu);
-    for (int64_t u = 0; u < nu; ++u) order[u] = u;
-    std::vector<std::pair<int64_t, int64_t>> gcost;   // (group, total cost)
-    for (int64_t u = 0; u < nu; ++u) {
-      if (gcost.empty() || gcost.back().first != units[u].group) gcost.push_back({units[u].group, 0});
-      gcost.back().second += cost[u];
-    }
-    std::vector<int64_t> gtotal(nu);
+    std::vector<int64_t> gmax(nu);
     {
+      std::vector<std::pair<int64_t, int64_t>> gm;   // (group, largest unit cost)
+      for (int64_t u = 0; u < nu; ++u) {
+        if (gm.empty() || gm.back().first != units[u].group) gm.push_back({units[u].group, 0});
+        gm.back().second = std::max(gm.back().second, cost[u]);
+      }
       size_t gi = 0;
       for (int64_t u = 0; u < nu; ++u) {
-        while (gcost[gi].first != units[u].group) ++gi;
-        gtotal[u] = gcost[gi].second;
+        while (gm[gi].first != units[u].group) ++gi;
+        gmax[u] = gm[gi].second;
       }
     }
-    // (descending group total, group, descending cost, index): the index makes the order
-    // total, so a plain sort gives the stable order
+    // (descending largest unit of the group, group, descending cost, index): the index makes
+    // the order total, so a plain sort gives the stable order
     struct Key {
-      int64_t gt, grp, c, u;
+      int64_t gm, grp, c, u;
     };
     std::vector<Key> keys(nu);
-    for (int64_t u = 0; u < nu; ++u) keys[u] = {-gtotal[u], units[u].group, -cost[u], u};
+    for (int64_t u = 0; u < nu; ++u) keys[u] = {-gmax[u], units[u].group, -cost[u], u};
     std::sort(keys.begin(), keys.end(), [](const Key& a, const Key& b) {
-      if (a.gt != b.gt) return a.gt < b.gt;
+      if (a.gm != b.gm) return a.gm < b.gm;
       if (a.grp != b.grp) return a.grp < b.grp;
       if (a.c != b.c) return a.c < b.c;
       return a.u < b.u;
     });
-    for (int64_t i = 0; i < nu; ++i) order[i] = keys[i].u;
     const int32_t ctas = int32_t(std::min<int64_t>(grid, nu));
     // Min-heap of (load, cta): each unit goes to the least-loaded CTA (lowest index on ties),
     // whose load then grows -- one sift-down per unit instead of a pop and a push.
@@ -199,7 +202,8 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
     heap.resize(static_cast<size_t>(ctas));
     for (int32_t c = 0; c < ctas; ++c) heap[size_t(c)] = {0, c};   // already a heap
     pieces.reserve(size_t(nu));
-    for (int64_t u : order) {
+    for (const Key& k : keys) {
+      const int64_t u = k.u;
       Load& top = heap[0];
       pieces.push_back({int32_t(u), 0, int32_t(nb[u]), top.second});
       npieces[u] = 1;
@@ -228,6 +232,15 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
       pieces.swap(sorted);
     }
     num_ctas = ctas;
+  };
+
+  // The largest CTA load of the current pieces (block costs plus the per-piece overhead).
+  auto max_load = [&]() -> int64_t {
+    std::vector<int64_t> load(size_t(std::max(num_ctas, 0)), 0);
+    for (const Piece& pc : pieces) load[size_t(pc.cta)] += int64_t(pc.nblk) * units[size_t(pc.unit)].w + ovh;
+    int64_t mx = 0;
+    for (int64_t l : load) mx = std::max(mx, l);
+    return mx;
   };
 
   // Greedy fill of CTAs with capacity q (block costs + overhead per piece), in unit order;
@@ -304,7 +317,23 @@ int schedule(const rae_config& cfg, int32_t kind, const std::vector<Unit>& units
     int64_t prow = 0;
     for (int64_t u = 0; u < nu; ++u)
       if (npieces[u] > 1) prow += int64_t(npieces[u]) * units[u].rows;
-    if (prow > cfg.max_partial_rows || prow > max_merge_rows(cfg)) lpt();
+    if (prow > cfg.max_partial_rows || prow > max_merge_rows(cfg)) {
+      lpt();
+    } else if (lpt_slack_pct > 0) {
+      // Whole units win whenever their busiest CTA is within lpt_slack_pct of the split
+      // schedule's: they need no partials or merges, and the units of a group run side by
+      // side instead of one after another on one CTA (their K/V read once, through L2).
+      const int64_t split_max = max_load();
+      std::vector<Piece> split_pieces = pieces;
+      std::vector<int32_t> split_np = npieces;
+      const int32_t split_ctas = num_ctas;
+      lpt();
+      if (max_load() * 100 > split_max * (100 + lpt_slack_pct)) {
+        pieces.swap(split_pieces);
+        npieces.swap(split_np);
+        num_ctas = split_ctas;
+      }
+    }
   }
 
   if (int64_t(pieces.size()) > cfg.max_tiles)
@@ -491,8 +520,12 @@ int build_paged_plan(const rae_config& cfg, const int32_t* qo_indptr,
   Schedule sc;
   // The decode kernel is HBM bound and short: an even split of the bytes over the grid
   // matters more than the small merge it costs.
-  rc = simt ? schedule(cfg, kind, units, kSimtChunkKeys, 2, g, 64, &sc, err)
-            : schedule(cfg, kind, units, kTcBlockKeys, swap ? 1 : kTcStep, g, 4, &sc, err);
+  // The tensor-core kernel prefers whole units within 15 % of the split schedule's balance
+  // (measured on the packed multi-token and causal chunked-prefill workloads: 20 % faster
+  // calls with busiest CTAs 6 % and 2 % above the split schedule's).
+  rc = simt ? schedule(cfg, kind, units, kSimtChunkKeys, 2, g, 64, 0, &sc, err)
+       : swap ? schedule(cfg, kind, units, kTcBlockKeys, 1, g, 4, 0, &sc, err)
+              : schedule(cfg, kind, units, kTcBlockKeys, kTcStep, g, 4, kTcLptSlackPct, &sc, err);
   if (rc) return rc;
   rc = emit_image(sc, qo_indptr, batch + 1, kv_len, batch, kv_page_indptr, batch + 1,
                   kv_page_indices, nnz, image, image_words, out, err);
@@ -555,7 +588,7 @@ int build_ragged_plan(const rae_config& cfg, const int32_t* cu_q, const int32_t*
   out->rows_max = 0;
   for (const Unit& u : units) out->rows_max = std::max(out->rows_max, u.rows);
   Schedule sc;
-  rc = schedule(cfg, kKindTcRagged, units, kTcBlockKeys, kTcStep, g, 4, &sc, err);
+  rc = schedule(cfg, kKindTcRagged, units, kTcBlockKeys, kTcStep, g, 4, kTcLptSlackPct, &sc, err);
   if (rc) return rc;
   rc = emit_image(sc, cu_q, num_spans + 1, kv, num_spans + 1, nullptr, 0, nullptr, 0, image,
                   image_words, out, err);

@@ -77,9 +77,10 @@ def test_two_span_cross_multitoken_shapes():
     assert_close(out, oracle_ragged(case), what="cross multitoken")
 
 
-@pytest.mark.parametrize("bs,sms", [(256, 3), (0, 5)])
+@pytest.mark.parametrize("bs,sms", [(256, 8), (256, 12), (0, 5), (0, 12)])
 def test_forced_splits_ragged(bs, sms):
-    """A small grid over few long units cuts some units' keys: split tiles plus the merge."""
+    """A grid with more CTAs than whole units balance over cuts some units' keys: split
+    tiles plus the merge."""
     case = inputs.ragged_case(130, span_lens=[1500, 700], num_qo_heads=1, num_kv_heads=1,
                               head_dim=128, block_size=bs)
     out, plan, *_ = run_ragged(case, num_sms=sms)

@@ -370,11 +370,15 @@ def test_missing_library_fails_loudly():
 
 def test_tensor_core_fill_does_not_overshoot_a_cta_by_a_block():
     """The contiguous fill closes a CTA when not one more key block fits in its capacity, so
-    on the packed multi-token workload no CTA carries more than one block's cost above the
-    mean (block costs 16 or 17, 16 per tile)."""
-    c = inputs.workload(3)
-    p = plan_paged_host(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages,
-                        num_qo_heads=32, num_kv_heads=8, head_dim=128, page_size=16)
+    no CTA carries more than one block's cost above the mean (block costs 16 or 17, 16 per
+    tile).  Few long units (2 requests x 8 KV heads over 30 000-key contexts) need that fill:
+    whole units would leave most of the 148 CTAs idle."""
+    case = inputs.paged_case(7, q_lens=[64, 40], ctx_lens=[30000, 21000], num_qo_heads=32,
+                             num_kv_heads=8, head_dim=128, page_size=16)
+    p = plan_paged_host(case.qo_indptr, case.kv_page_indptr, case.kv_page_indices, case.kv_len,
+                        case.num_pages, num_qo_heads=32, num_kv_heads=8, head_dim=128,
+                        page_size=16, num_sms=148)
+    assert p["raw"].kind == 2 and p["raw"].num_merge_rows > 0
     t, cp = p["tiles"], p["cta_ptr"]
     tpt = 128 // 4
     load = []
@@ -385,3 +389,18 @@ def test_tensor_core_fill_does_not_overshoot_a_cta_by_a_block():
             s += nb * (17 if int(t[i, 3]) > tpt else 16) + 16
         load.append(s)
     assert max(load) <= np.mean(load) + 17, (max(load), np.mean(load))
+
+
+def test_tensor_core_plans_prefer_whole_units_when_balanced():
+    """Whole units (no splits, a group's query chunks side by side) are chosen for the packed
+    multi-token and chunked-prefill workloads, whose busiest CTA stays within 15 % of the
+    split schedule's."""
+    c = inputs.workload(3)
+    p = plan_paged_host(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages,
+                        num_qo_heads=32, num_kv_heads=8, head_dim=128, page_size=16)
+    assert p["raw"].num_merge_rows == 0 and p["raw"].num_ctas == 148
+    c = inputs.causal_chunked_prefill()
+    p = plan_paged_host(c.qo_indptr, c.kv_page_indptr, c.kv_page_indices, c.kv_len, c.num_pages,
+                        num_qo_heads=c.num_qo_heads, num_kv_heads=c.num_kv_heads,
+                        head_dim=c.head_dim, page_size=c.page_size, causal=True)
+    assert p["raw"].num_merge_rows == 0 and p["raw"].num_ctas == 148
