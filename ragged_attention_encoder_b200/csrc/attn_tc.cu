@@ -34,6 +34,10 @@ constexpr int kTcThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kStages = 2;
+// Q tiles sit in a ring of three slots: the next unit's first Q tile loads while the current
+// unit still runs (its slot was released by the unit before), the second as soon as the
+// current unit's last S of tile 0 has read that tile's slot.
+constexpr int kQSlots = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kChunkBytes = 128 * 128;   // 128 rows x 64 bf16 (one 128-byte swizzle span)
 
@@ -42,18 +46,19 @@ template <int D>
 struct TcLayout {
   static constexpr int CH = D / 64;
   static constexpr int TILE = CH * kChunkBytes;   // bytes of a 128-row Q, K or V tile
-  static constexpr int Q_OFF = 0;                  // Q0, Q1
-  static constexpr int K_OFF = 2 * TILE;
+  static constexpr int Q_OFF = 0;                  // the ring of Q tile slots
+  static constexpr int K_OFF = kQSlots * TILE;
   static constexpr int V_OFF = K_OFF + kStages * TILE;
   static constexpr int BAR_OFF = V_OFF + kStages * TILE;
   static constexpr int SMEM = BAR_OFF + 512 + 1024;   // barriers + alignment slack
+  static_assert(SMEM <= 232448, "shared memory of one CTA (227 KB)");
   // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 after it.
   static __device__ __forceinline__ constexpr uint32_t s_col(int qt) { return uint32_t(qt) * 128u; }
   static __device__ __forceinline__ constexpr uint32_t o_col(int qt) { return 256u + uint32_t(qt) * D; }
 };
 
 struct TcBars {
-  uint64_t q_full, q_empty, fin;
+  uint64_t q_full[kQSlots], q_empty[kQSlots], fin;
   uint64_t merge_in, merge_out;   // split-unit arrival protocol (softmax warps)
   int merge_flag;
   uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
@@ -142,8 +147,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
   const Geometry& geo = p.geo;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bar.q_full, 1);
-    mbar_init(&bar.q_empty, 1);
+    for (int i = 0; i < kQSlots; ++i) {
+      mbar_init(&bar.q_full[i], 1);
+      mbar_init(&bar.q_empty[i], 1);
+    }
     mbar_init(&bar.fin, 1);
     mbar_init(&bar.merge_in, 8);
     mbar_init(&bar.merge_out, 1);
@@ -193,7 +200,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
     const uint64_t pol_q = policy_evict_first();
     const uint64_t pol_kv = policy_evict_last();
     const uint32_t q_tile_bytes = uint32_t(L::CH) * 64u * 2u * uint32_t(g * tpt);
-    uint32_t q_use = 0, kv_use = 0;
+    uint32_t q_cnt = 0, kv_use = 0;   // Q tiles armed; K/V blocks
     bool ok = true;
     for (int t = t_begin; t < t_end && ok; ++t) {
       const Tile tile = plan.tiles[t];
@@ -201,19 +208,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       if (n == 0) continue;
       const bool has1 = tile.qn > tpt;
       if (lane == 0) {
-        if (q_use > 0 && !wait_bounded(&bar.q_empty, (q_use - 1) & 1, wc, 201)) {
-          ok = false;
-        } else {
-          mbar_arrive_expect_tx(&bar.q_full, q_tile_bytes * (has1 ? 2u : 1u));
-          for (int qt = 0; qt < (has1 ? 2 : 1); ++qt)
-            for (int c = 0; c < L::CH; ++c)
-              tma_load_3d(smem + L::Q_OFF + qt * L::TILE + c * kChunkBytes, &p.maps.q, &bar.q_full,
-                          c * 64, tile.kv_head * g, tile.q0 + qt * tpt, pol_q);
+        for (int qt = 0; qt < (has1 ? 2 : 1); ++qt) {
+          const int qs = int(q_cnt % kQSlots);
+          if (q_cnt >= uint32_t(kQSlots) &&
+              !wait_bounded(&bar.q_empty[qs], ((q_cnt / kQSlots) - 1) & 1, wc, 201)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar.q_full[qs], q_tile_bytes);
+          for (int c = 0; c < L::CH; ++c)
+            tma_load_3d(smem + L::Q_OFF + qs * L::TILE + c * kChunkBytes, &p.maps.q, &bar.q_full[qs],
+                        c * 64, tile.kv_head * g, tile.q0 + qt * tpt, pol_q);
+          ++q_cnt;
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
+      q_cnt = __shfl_sync(0xffffffffu, q_cnt, 0);
       if (!ok) break;
-      ++q_use;
       const int32_t* pages = p.paged ? plan.d + plan.c[tile.req] : nullptr;
       const int32_t kv_base = p.paged ? 0 : plan.b[tile.req];
       for (int j = 0; j < n; ++j, ++kv_use) {
@@ -283,9 +294,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
                int64_t(global_timer_ns() - t0) < lim) {
         }
       }
-      if (q_use > 0) {
+      for (uint32_t c = q_cnt > uint32_t(kQSlots) ? q_cnt - kQSlots : 0; c < q_cnt; ++c) {
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(&bar.q_full, (q_use - 1) & 1) && int64_t(global_timer_ns() - t0) < lim) {
+        while (!mbar_try_wait(&bar.q_full[c % kQSlots], (c / kQSlots) & 1) &&
+               int64_t(global_timer_ns() - t0) < lim) {
         }
       }
     }
@@ -294,7 +306,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-      uint32_t q_use = 0, kv_use = 0;
+      uint32_t q_cnt = 0, kv_use = 0;
       uint32_t pv_cnt0 = 0, pv_cnt1 = 0, o_tiles0 = 0, o_tiles1 = 0;
       bool ok = true;
       for (int t = t_begin; t < t_end && ok; ++t) {
@@ -302,8 +314,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         const int n = tile_blocks(tile);
         if (n == 0) continue;
         const bool has1 = tile.qn > tpt;
-        if (!wait_bounded(&bar.q_full, q_use & 1, wc, 214)) { ok = false; break; }
-        ++q_use;
+        // Q slot of each tile of this unit, and its shared-memory address
+        const int qs[2] = {int(q_cnt % kQSlots), int((q_cnt + 1) % kQSlots)};
+        const uint32_t qa[2] = {sbase + L::Q_OFF + qs[0] * L::TILE, sbase + L::Q_OFF + qs[1] * L::TILE};
+        for (int qt = 0; qt < (has1 ? 2 : 1) && ok; ++qt)
+          ok = wait_bounded(&bar.q_full[qs[qt]], ((q_cnt + qt) / kQSlots) & 1, wc, 214);
+        if (!ok) break;
+        q_cnt += has1 ? 2 : 1;
         // Prologue: S of block 0 for both tiles.
         {
           const int s = kv_use % kStages;
@@ -312,12 +329,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
 #pragma unroll
           for (int qt = 0; qt < 2; ++qt) {
             if (qt == 1 && !has1) break;
-            mma_s<D>(tmem + L::s_col(qt), sbase + L::Q_OFF + qt * L::TILE,
-                     sbase + L::K_OFF + s * L::TILE, idesc_qk);
+            mma_s<D>(tmem + L::s_col(qt), qa[qt], sbase + L::K_OFF + s * L::TILE, idesc_qk);
             umma_commit(&bar.s_full[qt]);
+            if (n == 1) umma_commit(&bar.q_empty[qs[qt]]);   // this tile's last S
           }
           umma_commit(&bar.k_empty[s]);
-          if (n == 1) umma_commit(&bar.q_empty);
         }
         for (int j = 0; j < n && ok; ++j) {
           const uint32_t use = kv_use + j;
@@ -342,17 +358,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
             umma_commit(&bar.pv_done[qt]);
             if (qt) ++pv_cnt1; else ++pv_cnt0;
             if (more) {   // after P_qt(j) was consumed (the tensor pipe runs in issue order)
-              mma_s<D>(tmem + L::s_col(qt), sbase + L::Q_OFF + qt * L::TILE,
-                       sbase + L::K_OFF + s1 * L::TILE, idesc_qk);
+              mma_s<D>(tmem + L::s_col(qt), qa[qt], sbase + L::K_OFF + s1 * L::TILE, idesc_qk);
               umma_commit(&bar.s_full[qt]);
+              if (j + 2 == n) umma_commit(&bar.q_empty[qs[qt]]);   // this tile's last S
             }
           }
           if (!ok) break;
           umma_commit(&bar.v_empty[s]);
-          if (more) {
-            umma_commit(&bar.k_empty[s1]);
-            if (j + 2 == n) umma_commit(&bar.q_empty);
-          }
+          if (more) umma_commit(&bar.k_empty[s1]);
         }
         kv_use += n;
         ++o_tiles0;
