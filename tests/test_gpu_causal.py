@@ -123,6 +123,22 @@ def test_paged_causal_with_forced_splits(num_sms, qmax):
     assert_close(out, ref, what=f"causal split sms={num_sms} q<={qmax}")
 
 
+@pytest.mark.parametrize("kv_lens", [[140, 150, 260], [200, 385, 300]])
+def test_one_tile_unit_rows_whose_limit_ends_in_the_first_block(kv_lens):
+    """One query tile over two or three key blocks, causal: the early queries' limits fall
+    before the second block, so every key of that block is masked for those rows."""
+    q_lens = [30, 32, 25]
+    case = _stream_case(335 + sum(kv_lens), q_lens, kv_lens, 16, 4, 128, 16)
+    ctx = Context(16, 4, 128, 16)
+    kp, vp = _write_then_append(case, ctx)
+    out, plan = _run(case, ctx, kp, vp)
+    assert plan.kernel_kind == 2
+    rk, rv = _oracle_pools(case)
+    ref = oracle.paged_causal_attention(case.q, rk, rv, case.qo_indptr, case.kv_page_indptr,
+                                        case.kv_page_indices, case.kv_len)
+    assert_close(out, ref, what=f"causal one tile {kv_lens}")
+
+
 def test_prefill_whole_stream():
     """qlen == kv_len: the whole stream is new (a prompt's first step)."""
     lens = [1, 128, 300, 77]

@@ -213,6 +213,25 @@ def test_empty_context_gives_zero():
     assert_close(out, oracle_paged(case), what="empty ctx tc")
 
 
+@pytest.mark.parametrize("ctx_lens,split_sms", [([129, 256], 7), ([257, 300, 383], 11),
+                                                ([129, 1000, 513, 640, 900], 20)])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("split", [False, True])
+def test_one_tile_units_over_several_key_blocks(ctx_lens, split_sms, d, split):
+    """Units with one 128-row query tile over two to eight key blocks: even and odd block
+    counts, a partial last block, pools of NaN around the pages, with and without cuts inside
+    the keys."""
+    q_lens = [17 + 5 * i for i in range(len(ctx_lens))]      # 68..148 rows at GQA 4
+    case = inputs.paged_case(700 + d + len(ctx_lens), q_lens=q_lens, ctx_lens=ctx_lens,
+                             num_qo_heads=16, num_kv_heads=4, head_dim=d, page_size=16)
+    cap = {"num_sms": split_sms} if split else {}
+    out, plan, *_ = run_paged(case, **cap)
+    assert plan.kernel_kind == 2
+    if split:
+        assert plan.num_merge_rows > 0    # this grid cuts units inside their keys
+    assert_close(out, oracle_paged(case), what=f"paired {ctx_lens} d={d} split={split}")
+
+
 @pytest.mark.parametrize("num_sms,qmax", [(2, 1), (3, 1), (5, 1), (6, 50), (8, 50), (16, 50)])
 def test_forced_splits_agree_with_oracle_and_unsplit(num_sms, qmax):
     case = inputs.paged_case(70 + num_sms + qmax, q_lens=(1, qmax, 3), ctx_lens=(300, 3000, 3),
