@@ -134,6 +134,13 @@ __device__ __noinline__ void rescale_o(uint32_t o_addr, float f) {
   }
 }
 
+// The split merge, kept out of line so that its registers do not add to the softmax loop's.
+template <int D>
+__device__ __noinline__ void merge_unit(const Tile& tile, const Geometry& geo, const float* part_o,
+                                        const float* part_lse, __nv_bfloat16* out) {
+  merge_split_unit<D, 8>(tile, geo, tile.kv_head * geo.g, geo.g, part_o, part_lse, out, threadIdx.x, 256);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
   using L = TcLayout<D>;
@@ -390,7 +397,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
     uint32_t kv_use = 0, s_cnt = 0, pv_cnt = 0, split_seen = 0;
     bool ok = true;
     for (int t = t_begin; t < t_end && ok; ++t) {
-      const Tile tile = plan.tiles[t];
+      const Tile& tile = plan.tiles[t];
       const int n = tile_blocks(tile);
       const bool has1 = tile.qn > tpt;
       if (qt == 1 && !has1) {
@@ -398,7 +405,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         if (tile.part >= 0 &&
             split_unit_complete(plan.counters, tile, &bar.merge_in, &bar.merge_out, &bar.merge_flag,
                                 split_seen++, false, lane, wc, &ok))
-          merge_split_unit<D, 8>(tile, geo, tile.kv_head * geo.g, geo.g, p.part_o, p.part_lse, p.out, threadIdx.x, 256);
+          merge_unit<D>(tile, geo, p.part_o, p.part_lse, p.out);
         continue;
       }
       const int tok = qt * tpt + tok_in_tile;     // token index within the work tile
@@ -566,7 +573,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       if (split &&
           split_unit_complete(plan.counters, tile, &bar.merge_in, &bar.merge_out, &bar.merge_flag,
                               split_seen++, threadIdx.x == 0, lane, wc, &ok))
-        merge_split_unit<D, 8>(tile, geo, tile.kv_head * geo.g, geo.g, p.part_o, p.part_lse, p.out, threadIdx.x, 256);
+        merge_unit<D>(tile, geo, p.part_o, p.part_lse, p.out);
     }
   }
 
