@@ -43,7 +43,9 @@ struct SimtCfg {
   static constexpr int ITERS = kSimtChunkKeys / KPI;
   static constexpr int CHUNK_ELEMS = kSimtChunkKeys * D;
   static constexpr int CHUNK_BYTES = CHUNK_ELEMS * 2;
-  static constexpr int NST = D == 64 ? 6 : 3;       // stages in the ring
+  // Stages in the ring: at d = 64 five 16 KB stages per CTA (two CTAs per SM) streamed
+  // faster than four, six or seven.
+  static constexpr int NST = D == 64 ? 5 : 3;
   static constexpr int STAGE_ELEMS = 2 * kSimtConsumers * CHUNK_ELEMS;   // K chunks, V chunks
 };
 
