@@ -77,6 +77,7 @@ struct TcParams {
   int* err;
   float scale_log2;
   int32_t paged;
+  int32_t wide_stores;   // out and the partials are 32-byte aligned: one sector per store
   int64_t timeout_ns;
 };
 
@@ -546,20 +547,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
           for (int e = 0; e < 32; ++e) ov[e] = 0u;
         }
         if (!row_ok) continue;
+        // A thread writes its own row: with 32-byte stores every store fills whole sectors
+        // (the rows of a warp are Hq * d elements apart).
         if (!split) {
           uint32_t pkd[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             pkd[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t(q_tok) * geo.hq + head) * D + c * 32);
+          __nv_bfloat16* row = p.out + (int64_t(q_tok) * geo.hq + head) * D + c * 32;
+          if (p.wide_stores) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
+            for (int e = 0; e < 2; ++e)
+              st_global_v8(row + 16 * e, pkd[8 * e], pkd[8 * e + 1], pkd[8 * e + 2], pkd[8 * e + 3],
+                           pkd[8 * e + 4], pkd[8 * e + 5], pkd[8 * e + 6], pkd[8 * e + 7]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(row);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
+          }
         } else {
-          float4* dst = reinterpret_cast<float4*>(p.part_o + int64_t(tile.part + urow) * D + c * 32);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
-                                 __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * inv);
+          float* row = p.part_o + int64_t(tile.part + urow) * D + c * 32;
+          if (p.wide_stores) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              st_global_v8(row + 8 * e, ov[8 * e], ov[8 * e + 1], ov[8 * e + 2], ov[8 * e + 3], ov[8 * e + 4],
+                           ov[8 * e + 5], ov[8 * e + 6], ov[8 * e + 7]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(row);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dst[e] = make_uint4(ov[4 * e], ov[4 * e + 1], ov[4 * e + 2], ov[4 * e + 3]);
+          }
         }
       }
       if (split && row_ok) p.part_lse[tile.part + urow] = l > 0.f ? m + fast_log2(l) : -INFINITY;
@@ -601,6 +620,7 @@ cudaError_t launch_attn_tc(const DevPlan& plan, const Geometry& geo, bool paged,
   prm.err = err;
   prm.scale_log2 = scale_log2;
   prm.paged = paged ? 1 : 0;
+  prm.wide_stores = ((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(part_o)) & 31) == 0;
   prm.timeout_ns = timeout_ns;
   cudaError_t e;
   if (geo.d == 128) {
