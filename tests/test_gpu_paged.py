@@ -244,6 +244,31 @@ def test_forced_splits_agree_with_oracle_and_unsplit(num_sms, qmax):
     assert_close(out_full, ref, what="unsplit")
 
 
+@pytest.mark.parametrize("num_sms,split", [(5, False), (148, True)])
+def test_output_aligned_to_16_bytes_only(num_sms, split):
+    """An output whose address is 16- but not 32-byte aligned takes the kernels' 16-byte store
+    path (32-byte stores need 32-byte alignment) and gives the same result, with and without
+    split partials."""
+    case = inputs.paged_case(91, q_lens=[20, 33, 7], ctx_lens=[300, 1000, 129], num_qo_heads=16,
+                             num_kv_heads=4, head_dim=128, page_size=16)
+    ctx = context_for(case, num_sms=num_sms)
+    kp, vp = gpu_pools(case, ctx)
+    plan = ctx.plan_paged(case.qo_indptr, case.kv_page_indptr, case.kv_page_indices, case.kv_len,
+                          case.num_pages)
+    assert plan.kernel_kind == 2
+    assert (plan.num_merge_rows > 0) == split
+    q = case.q.cuda()
+    buf = torch.full((q.numel() + 16,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = buf[8:8 + q.numel()].view_as(q)
+    assert out.data_ptr() % 32 == 16
+    ctx.run_paged(plan, q, kp, vp, out)
+    torch.cuda.synchronize()
+    ctx.check_device_status()
+    assert_close(out, oracle_paged(case), what=f"16-byte aligned out, sms={num_sms}")
+    aligned, *_ = run_paged(case, num_sms=num_sms)
+    assert torch.equal(out.view(torch.int16), aligned.view(torch.int16))
+
+
 def test_explicit_scale():
     case = inputs.paged_case(81, q_lens=[3, 20], ctx_lens=[100, 257], num_qo_heads=8,
                              num_kv_heads=2, head_dim=64, page_size=16)
