@@ -66,6 +66,7 @@ struct PwParams {
   int32_t kchunks;                    // H / 64
   int32_t n_half;                     // Hkv * d
   int32_t hkv, d, page_size;
+  int32_t wide_stores;                // both pools 32-byte aligned: one whole sector per store
 };
 
 template <int BN, int STAGES>
@@ -202,9 +203,19 @@ __global__ void __launch_bounds__(kPwThreads) project_write_kernel(const __grid_
         for (int j = 0; j < 16; ++j)
           pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]) + bf16lo_to_f32(bw[j]),
                               __uint_as_float(v[2 * j + 1]) + bf16hi_to_f32(bw[j]));
-        uint4* dst = reinterpret_cast<uint4*>(pool + (dst_row + int64_t(h) * p.page_size) * p.d + e0);
+        // A thread's 64 bytes: with 32-byte stores each fills a whole sector (the rows of a
+        // warp are d elements apart).
+        __nv_bfloat16* row = pool + (dst_row + int64_t(h) * p.page_size) * p.d + e0;
+        if (p.wide_stores) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          for (int j = 0; j < 2; ++j)
+            st_global_v8(row + 16 * j, pk[8 * j], pk[8 * j + 1], pk[8 * j + 2], pk[8 * j + 3], pk[8 * j + 4],
+                         pk[8 * j + 5], pk[8 * j + 6], pk[8 * j + 7]);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(row);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        }
       }
     }
   }
@@ -256,6 +267,7 @@ cudaError_t launch_project_write(const ProjectWriteArgs& a, cudaStream_t stream)
   prm.hkv = a.geo.hkv;
   prm.d = a.geo.d;
   prm.page_size = a.geo.page_size;
+  prm.wide_stores = ((reinterpret_cast<uintptr_t>(a.k_pool) | reinterpret_cast<uintptr_t>(a.v_pool)) & 31) == 0;
   // (the weight maps' box height must be project_write_tile_cols(n_half))
   if (project_write_tile_cols(prm.n_half) != 128) return launch_bn<PW_BN_WIDE, PW_STAGES_WIDE>(prm, a.m, stream);
   return launch_bn<128, 3>(prm, a.m, stream);
