@@ -958,8 +958,8 @@ def run_counters(args):
     plainly, then under ncu with a handful of metrics on one launch (the second of its
     kernel; `--clock-control none`).  Writes profiles/counters.json."""
     ncu = os.environ.get("NCU", "ncu")
-    outdir = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) \
-        else tempfile.mkdtemp()
+    outdir = os.environ.get("RAE_NCU_LOG_DIR") or tempfile.mkdtemp()   # raw ncu CSVs
+    os.makedirs(outdir, exist_ok=True)
     entries = []
     for case_id, (workload, kernel, source) in PROFILE_CASES.items():
         cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--profile-case", str(case_id),
