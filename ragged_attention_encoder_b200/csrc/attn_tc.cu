@@ -363,7 +363,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
             tc_fence_after();
             mma_pv<D>(tmem + L::o_col(qt), tmem + L::s_col(qt), sbase + L::V_OFF + s * L::TILE,
                       idesc_pv, j == 0);
-            umma_commit(&bar.pv_done[qt]);
+            // The unit's last P.V is signalled for the epilogue; an earlier one needs no signal
+            // of its own: S of the next block is issued after it, so s_full covers it.
+            if (!more) umma_commit(&bar.pv_done[qt]);
             if (qt) ++pv_cnt1; else ++pv_cnt0;
             if (more) {   // after P_qt(j) was consumed (the tensor pipe runs in issue order)
               mma_s<D>(tmem + L::s_col(qt), qa[qt], sbase + L::K_OFF + s1 * L::TILE, idesc_qk);
@@ -495,10 +497,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         const float psum = f32x2_sum(ps[0]) + f32x2_sum(ps[1]);
         l = l * corr + psum;
         if (__any_sync(0xffffffffu, rescale)) {
-          // O holds the sum through block j-1 once P.V of block j-1 has completed.
-          ok = __all_sync(0xffffffffu, wait_bounded(&bar.pv_done[qt], (pv_cnt + j - 1) & 1, wc, 222));
-          if (!ok) break;
-          tc_fence_after();
+          // O holds the sum through block j-1: P.V of block j-1 was issued before S of block
+          // j, whose completion (s_full, waited for above) covers it.
           rescale_o<D>(lane_addr + o_col, corr);
         }
         tmem_wait_st();
@@ -526,13 +526,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       kv_use += n;
       // ---------------------------------------------------------------- epilogue
       const bool split = tile.part >= 0;
+      // pv_done completes once per unit of this tile (after its last P.V).
       if (!live) {
-        pv_cnt += n;
+        if (n > 0) ++pv_cnt;
       } else {
       if (n > 0) {
-        ok = __all_sync(0xffffffffu, wait_bounded(&bar.pv_done[qt], (pv_cnt + n - 1) & 1, wc, 224));
+        ok = __all_sync(0xffffffffu, wait_bounded(&bar.pv_done[qt], pv_cnt & 1, wc, 224));
         if (!ok) break;
-        pv_cnt += n;
+        ++pv_cnt;
         tc_fence_after();
       }
       const float inv = l > 0.f ? 1.f / l : 0.f;
